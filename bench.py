@@ -1,0 +1,394 @@
+"""Benchmark: 200K-token prefill of one 8-layer group with index sharing.
+
+One step = layer_group_forward over 8 layers with pattern FSSSFSSS (one
+indexer per four layers): 2 fused indexer + top-k launches and 8 sparse
+attention launches on a 200000-token sequence (H_I=32, d_I=128, top-2048,
+GQA 32 query / 4 KV heads, d=128, bf16; output bf16).  The same group with
+pattern FFFFFFFF (every layer indexes) is timed alongside for the indexer
+time ratio.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torchrun: every rank runs its own independent sequence
+(replicas, weak scaling; the path has no cross-GPU exchange), the step
+time is the max over ranks and `value` counts the tokens of all ranks.
+Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on
+the host cores on a bounded sample of rows of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tok/s at 200K ctx (indexer+top-k+sparse attn), % roofline"
+L, H_I, D_I, TOPK = 200000, 32, 128, 2048
+HQ, HKV, DH = 32, 4, 128
+PATTERN = "FSSSFSSS"
+ALL_F = "FFFFFFFF"
+N_LAYERS = 8
+WORKLOAD = (f"prefill L={L}, batch 1, 8 layers {PATTERN} (1 indexer per 4 layers; all-F timed too), "
+            f"indexer H_I={H_I} d_I={D_I} bf16 top-{TOPK}, sparse attention GQA {HQ}Q/{HKV}KV d={DH} bf16, "
+            f"bf16 output")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------- algorithmic work
+def gathered_rows(L_, k):
+    """sum_t min(k, t+1): KV rows one attention launch gathers per KV head."""
+    return k * (k + 1) // 2 + max(0, L_ - k) * k
+
+
+def attn_bytes(L_=L, k=TOPK):
+    return gathered_rows(L_, k) * HKV * (DH + DH) * 2
+
+
+def indexer_flops(L_=L):
+    return 2 * H_I * D_I * L_ * (L_ + 1) // 2
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index, path):
+        self.path = path
+        self.p = None
+        try:
+            self.f = open(path, "w")
+            self.p = subprocess.Popen(
+                ["nvidia-smi", f"--id={index}",
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from long_context_dsa_b200 import dsa, synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    hbm, bf16_burst, bf16_sus, peak_src = peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- inputs (seeded; each rank its own sequence)
+    gen = synth.StructuredIndexer("prefill200k", 1, L, H_I, D_I, r=32, base_std=1.0, noise_std=0.2,
+                                  device=dev, seed=1000 + rank)
+    layers = []
+    for l in range(N_LAYERS):
+        q, k, w = gen.layer(l)
+        Q, K, V = synth.attention_inputs("prefill200k", l, 1, L, L, HQ, HKV, DH, DH, device=dev, seed=1000 + rank)
+        layers.append({"q_I": q, "k_I": k, "w": w, "Q": Q, "K": K, "V": V,
+                       "O": torch.empty((1, L, HQ, DH), dtype=torch.bfloat16, device=dev)})
+    del gen
+    torch.cuda.synchronize()
+    shape = dsa.group_shape(1, L, 0, L, H_I, D_I, HQ, HKV, DH, DH, TOPK, o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((1, L, TOPK), dtype=torch.int32, device=dev))
+
+    def make_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * N_LAYERS)]
+        for e in evs:
+            e.record(stream)
+        return evs
+
+    def step(pattern, evs=None):
+        return dsa.layer_group_forward(shape, layers, pattern, cache, workspace=ws, events=evs)
+
+    for _ in range(args.warmup):
+        step(PATTERN)
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+
+    # ---- timed region: K steps of the shared-index group
+    step_evs = [make_events() for _ in range(args.steps)]
+    clk = ClockSampler(local_rank, os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
+                                                else ".", f"clocks_rank{rank}.csv"))
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    launches = 0
+    for i in range(args.steps):
+        st = step(PATTERN, step_evs[i])
+        launches += st.indexer_launches + st.attention_launches
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = clk.stop()
+    dsa.check_status(ws)
+    ms_local = t0.elapsed_time(t1)
+    idx_ms, attn_ms = [], []
+    for evs in step_evs:
+        for l in range(N_LAYERS):
+            if PATTERN[l] == "F":
+                idx_ms.append(evs[3 * l].elapsed_time(evs[3 * l + 1]))
+            attn_ms.append(evs[3 * l + 1].elapsed_time(evs[3 * l + 2]))
+
+    # ---- all-F group (indexer ratio), untimed for `value`
+    allf_evs = make_events()
+    step(ALL_F)
+    torch.cuda.synchronize()
+    allf_evs = make_events()
+    step(ALL_F, allf_evs)
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    allf_idx = [allf_evs[3 * l].elapsed_time(allf_evs[3 * l + 1]) for l in range(N_LAYERS)]
+    allf_step = allf_evs[0].elapsed_time(allf_evs[-1])
+
+    # ---- end to end through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, layers, shape, cache, ws, dev, stream)
+
+    # ---- max over ranks
+    ms = ms_local
+    if world > 1:
+        t = torch.tensor([ms_local], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    idx_avg = sum(idx_ms) / len(idx_ms)
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    value = world * L / (ms_per_step / 1e3)
+
+    abytes = attn_bytes()
+    iflops = indexer_flops()
+    t_idx = 2 * iflops / (bf16_sus * 1e12)
+    t_gather = N_LAYERS * abytes / (hbm * 1e9)
+    step_roof_s = max(t_idx, t_gather)
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded structured generator; no dataset or trained weights)",
+        "config": {"workload": WORKLOAD, "seq_len": L, "global_batch": world, "layers": N_LAYERS,
+                   "pattern": PATTERN, "topk": TOPK, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (q_I 1.6 GB, Q 1.6 GB per layer); no flush needed"},
+        "roofline": {
+            "bound": "hbm", "kernel": "sparse_attn_kernel (gathered K/V rows)",
+            "achieved": round(abytes / (attn_avg / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(abytes / (attn_avg / 1e3) / 1e9 / hbm, 4), "traffic": None,
+            "peak_source": f"{peak_src} hbm_gbs",
+            "algorithmic_bytes_per_launch": abytes, "avg_launch_ms": round(attn_avg, 3)},
+        "indexer_roofline": {
+            "bound": "tensor", "kernel": "indexer_topk_kernel (fused scores + top-k)",
+            "achieved": round(iflops / (idx_avg / 1e3) / 1e12, 1), "peak": bf16_sus, "unit": "TFLOP/s",
+            "frac": round(iflops / (idx_avg / 1e3) / 1e12 / bf16_sus, 4),
+            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel inside a long step)",
+            "frac_of_burst": round(iflops / (idx_avg / 1e3) / 1e12 / bf16_burst, 4),
+            "algorithmic_flops_per_launch": iflops, "avg_launch_ms": round(idx_avg, 3)},
+        "step_roofline": {"t_indexer_s": round(t_idx, 4), "t_gather_s": round(t_gather, 4),
+                          "bound_s": round(step_roof_s, 4),
+                          "frac": round(step_roof_s / (ms_per_step / 1e3), 4),
+                          "note": "max(indexer FLOPs at tensor peak, gathered bytes at HBM peak)"},
+        "index_sharing": {"all_f_step_ms": round(allf_step, 3), "shared_step_ms": round(ms_per_step, 3),
+                          "all_f_indexer_ms": round(sum(allf_idx), 3),
+                          "shared_indexer_ms": round(sum(idx_ms) / args.steps, 3),
+                          "indexer_time_ratio": round(sum(allf_idx) / (sum(idx_ms) / args.steps), 3)},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        out["e2e"] = e2e
+    return out
+
+
+def run_e2e(args, layers, shape, cache, ws, dev, stream):
+    """Same metric through layer_group_forward with host buffers: every step copies its inputs
+    host->device from pinned memory and reads every layer's output back."""
+    import torch
+    from long_context_dsa_b200 import dsa
+
+    names_f = ("q_I", "k_I", "w", "Q", "K", "V")
+    names_s = ("Q", "K", "V")
+    host_in, host_out = [], []
+    for l, Lh in enumerate(layers):
+        names = names_f if PATTERN[l] == "F" else names_s
+        host_in.append({n: torch.empty_like(Lh[n], device="cpu").pin_memory() for n in names})
+        for n in names:
+            host_in[-1][n].copy_(Lh[n])
+        host_out.append(torch.empty_like(Lh["O"], device="cpu").pin_memory())
+    h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    steps = max(1, min(args.steps, 2))
+
+    def one():
+        for l, Lh in enumerate(layers):
+            for n, t in host_in[l].items():
+                Lh[n].copy_(t, non_blocking=True)
+        dsa.layer_group_forward(shape, layers, PATTERN, cache, workspace=ws)
+        for l, Lh in enumerate(layers):
+            host_out[l].copy_(Lh["O"], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b) / steps
+    return {"value": round(L / (ms / 1e3), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms, 3),
+            "note": "pinned host inputs copied in and every layer's bf16 output read back inside the timed region"}
+
+
+# ------------------------------------------------------------ CPU oracle arm
+def oracle_sample(n_rows: int, seed: int = 0):
+    """Time the oracle on `n_rows` query rows of the workload (spread over t, last row included)
+    and extrapolate to the full step by algorithmic work.  Returns (tok/s, seconds, sample text, threads)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from long_context_dsa_b200 import synth
+
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[L - 1], rng.integers(0, L, n_rows - 1)]))
+    gen = synth.StructuredIndexer("prefill200k", 1, L, H_I, D_I, r=32, base_std=1.0, noise_std=0.2, seed=1000)
+    t_idx = t_att = 0.0
+    work_idx = work_att = 0.0
+    for l in range(N_LAYERS):
+        Q, K, V = synth.attention_inputs("prefill200k", l, 1, L, L, HQ, HKV, DH, DH, seed=1000)
+        if PATTERN[l] == "F":
+            q, k, w = gen.layer(l)
+            sel = {}
+            for t in rows:
+                a = time.perf_counter()
+                sc = oracle.indexer_scores(q[0, t:t + 1], k[0, :t + 1], w[0, t:t + 1], q_pos0=t)
+                sel[t] = oracle.topk_select(sc, TOPK, q_pos0=t)
+                t_idx += time.perf_counter() - a
+                work_idx += t + 1
+        for t in rows:
+            a = time.perf_counter()
+            oracle.sparse_attention(Q[0, t:t + 1], K[0], V[0], sel[t])
+            t_att += time.perf_counter() - a
+            work_att += min(TOPK, t + 1)
+    n_f = PATTERN.count("F")
+    # seconds per candidate key of one F layer, per gathered row of one layer
+    per_idx = t_idx / work_idx
+    per_att = t_att / work_att
+    total = per_idx * n_f * (L * (L + 1) / 2) + per_att * N_LAYERS * gathered_rows(L, TOPK)
+    threads = torch.get_num_threads()
+    sample = (f"{len(rows)} query rows (seeded, spread over t, last row included) through the {PATTERN} group: "
+              f"indexer+top-k on {n_f} F layers and attention on {N_LAYERS} layers; "
+              f"{t_idx + t_att:.1f} s measured, extrapolated by algorithmic work "
+              f"(sum of t+1 for the indexer, sum of min(k,t+1) for attention)")
+    return L / total, total, sample, threads, t_idx + t_att
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    vals, measured = [], 0.0
+    for i in range(args.warmup + args.steps):
+        v, total, sample, threads, meas = oracle_sample(args.ref_rows, seed=i)
+        if i >= args.warmup:
+            vals.append(v)
+            measured += meas
+    value = sum(vals) / len(vals)
+    return {"metric": METRIC, "impl": "reference", "value": round(value, 3), "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(L / value * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "seq_len": L, "pattern": PATTERN},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_gpu(args, rank, world, local_rank)
+    if rank == 0 and args.cpu_rows > 0:
+        v, total, sample, threads, meas = oracle_sample(args.cpu_rows)
+        out["cpu_baseline"] = {"value": round(v, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
+                               "sample": sample}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

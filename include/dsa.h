@@ -1,0 +1,246 @@
+/*
+ * dsa.h -- C ABI of libdsa.so: the DeepSeek-Sparse-Attention-style token
+ * indexer with cross-layer index reuse (IndexCache F/S layers; IndexShare,
+ * one indexer per four layers), for NVIDIA B200 (sm_100a).
+ *
+ * Sources the operations follow (Chinese web pages, cited by title and
+ * section):
+ *   [QbitAI]    QbitAI article on IndexCache (app.myzaker.com), sections
+ *               "IndexCache" and "GLM-5.2 已经用过了".
+ *   [Term]      earlyterms.com term page "IndexShare", definition.
+ *   [Explainer] "IndexShare 技术解读：4 层共享 indexer 如何把计算成本砍到三分之一"
+ *               (yun88.com), sections "稀疏注意力的隐性开销：indexer" and
+ *               "IndexShare 的共享机制：每 4 层一个 indexer".
+ *   [Linkstar]  "20万token压进10秒，清华这波操作让AI算力成本直接砍半"
+ *               (linkstar.cloud), sections on DSA's cost and on F/S layers
+ *               ("'偷懒'的艺术：相邻层其实在重复劳动").
+ *
+ * Conventions for every entry point:
+ *   - Return value is a status code (DSA_OK == 0).  No C++ exception
+ *     crosses the ABI and no kernel traps; device-detected errors are
+ *     recorded in the workspace status word and returned by
+ *     dsa_check_status().
+ *   - Tensor arguments are DEVICE pointers owned by the caller, row-major
+ *     and contiguous in the stated layout.  The library never allocates
+ *     or frees device memory and keeps no pointer after a call returns.
+ *   - Scratch memory is a caller-owned device `workspace` of at least the
+ *     size the matching *_workspace_size() query reports.  Its first 256
+ *     bytes are the status word; calls that share a workspace must not
+ *     overlap on the GPU.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream.
+ *   - Shapes are validated on the host before any launch; a rejected call
+ *     launches nothing and returns DSA_ERR_INVALID_ARG or
+ *     DSA_ERR_UNSUPPORTED with a message in dsa_last_error().
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define DSA_OK               0
+#define DSA_ERR_INVALID_ARG  1  /* bad shape, null pointer, bad pattern, small workspace */
+#define DSA_ERR_UNSUPPORTED  2  /* valid request this build has no kernel for            */
+#define DSA_ERR_CUDA         3  /* a CUDA runtime call or launch failed                  */
+#define DSA_ERR_TIMEOUT      4  /* a bounded device-side wait gave up (status word)      */
+#define DSA_ERR_DEVICE       5  /* a kernel rejected its data (status word), e.g. an
+                                   index outside [-1, n_kv) or a NaN score               */
+
+/* ---- element types --------------------------------------------------- */
+#define DSA_BF16  0
+#define DSA_E4M3  1   /* OCP fp8 E4M3 (bias 7, max 448, no infinities) */
+#define DSA_F32   2
+
+/* ---- device status word bits (dsa_check_status detail) ---------------- */
+#define DSA_STATUS_TIMEOUT    0x1   /* a bounded wait expired                  */
+#define DSA_STATUS_BAD_INDEX  0x2   /* sparse attention met an out-of-range idx */
+#define DSA_STATUS_NAN_SCORE  0x4   /* top-k met a NaN score                    */
+#define DSA_STATUS_OVERFLOW   0x8   /* a candidate buffer would have overflowed */
+
+/* Largest top-k this build selects. */
+#define DSA_TOPK_MAX 2048
+
+/* Thread-local text of the last error raised on this host thread. */
+DSA_API const char* dsa_last_error(void);
+
+/* Library ABI version (major*100 + minor). */
+DSA_API int dsa_version(void);
+
+/* Read the workspace status word (synchronises `stream`), clear it, and map
+ * it to a status code: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE.  If
+ * `bits` is non-NULL it receives the raw DSA_STATUS_* bits. */
+DSA_API int dsa_check_status(void* workspace, void* stream, int* bits);
+
+/* Zero the status word (asynchronous on `stream`). */
+DSA_API int dsa_reset_status(void* workspace, void* stream);
+
+/* ======================================================================
+ * idx_score_topk -- indexer scores + per-row top-k, fused (F layers).
+ *
+ * Operation ([QbitAI] §IndexCache: a light indexer before each attention
+ * layer picks the important tokens; [Term]: its work is "dot product +
+ * top-k"; the form below is the DeepSeek-Sparse-Attention lightning
+ * indexer):
+ *     score[b,i,s] = sum_h w[b,i,h] * ReLU(q_I[b,i,h,:] . k_I[b,s,:])
+ * for s = 0 .. q_pos0+i (query row i sits at absolute position q_pos0+i
+ * and sees itself).  fp8: q_I and k_I are E4M3 codes whose real values
+ * are code * q_scale[b,i,h] and code * k_scale[b,s].
+ * Selection: the `topk` largest scores per row, ties to the lower token
+ * index; a row with no more than `topk` candidates selects them all.
+ * The L x L score matrix is never written to memory.
+ *
+ * Layouts:
+ *   q_I     [B, n_q, H_I, d_I]  bf16 or e4m3 (dtype)
+ *   q_scale [B, n_q, H_I]       fp32, e4m3 only (else NULL)
+ *   k_I     [B, n_kv, d_I]      bf16 or e4m3
+ *   k_scale [B, n_kv]           fp32, e4m3 only (else NULL)
+ *   w       [B, n_q, H_I]       fp32
+ *   idx_out [B, n_q, topk]      int32: selected token indices of each row
+ *                               in ascending order, then -1 padding.
+ * Requires n_kv >= q_pos0 + n_q, 1 <= topk <= DSA_TOPK_MAX,
+ * H_I in {4, 8, 16, 32, 64}, d_I in {64, 128}.
+ * ====================================================================== */
+DSA_API int idx_score_topk_workspace_size(int B, int n_q, int q_pos0, int n_kv, int H_I, int d_I,
+                                  int topk, int dtype, size_t* bytes);
+DSA_API int idx_score_topk(const void* q_I, const float* q_scale, const void* k_I, const float* k_scale,
+                   const float* w, int dtype, int B, int n_q, int q_pos0, int n_kv,
+                   int H_I, int d_I, int topk, int32_t* idx_out,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* idx_scores -- the same indexer arithmetic without the selection: writes
+ * scores [B, n_q, n_kv] fp32 for the key tiles the fused kernel visits
+ * (s <= q_pos0+i exact, s > q_pos0+i within a visited tile -inf, other
+ * entries untouched).  For checking the scores themselves; it writes the
+ * full score matrix, so it is a test/debug path, not the product path.
+ * Workspace: 256 bytes (status word). */
+DSA_API int idx_scores(const void* q_I, const float* q_scale, const void* k_I, const float* k_scale,
+                       const float* w, int dtype, int B, int n_q, int q_pos0, int n_kv,
+                       int H_I, int d_I, float* scores, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* ======================================================================
+ * idx_topk_scores -- the top-k selection alone, on a given score array.
+ *
+ * Same selection code and rule as idx_score_topk; used to check the
+ * selection bit-exactly against a reference on identical scores.
+ *   scores  [rows, ld] fp32 (row i uses columns 0 .. q_pos0+i; ld >= n_kv)
+ *   idx_out [rows, topk] int32, layout as above.
+ * Scores in the causal range must not be NaN (DSA_STATUS_NAN_SCORE).
+ * ====================================================================== */
+DSA_API int idx_topk_scores_workspace_size(int rows, int q_pos0, int n_kv, int topk, size_t* bytes);
+DSA_API int idx_topk_scores(const float* scores, int rows, int q_pos0, int n_kv, int64_t ld, int topk,
+                    int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ======================================================================
+ * Index cache -- one int32 [rows, topk] buffer per layer group.
+ *
+ * [Linkstar] F/S layers: F layers keep the indexer and store the selected
+ * indices; S layers copy the most recent F layer's result and skip the
+ * indexer.  [QbitAI] §IndexCache: no extra GPU memory.  The cache is a
+ * host descriptor around ONE caller-owned device buffer; reading it
+ * launches nothing and copies nothing.
+ * ====================================================================== */
+typedef struct dsa_index_cache {
+    int32_t* buf;     /* caller-owned device buffer [rows, topk] */
+    int64_t rows;     /* B * n_q                                 */
+    int topk;
+    int writer;       /* layer that last wrote buf, -1 if none   */
+    int valid;        /* 1 once an F layer has written           */
+} dsa_index_cache;
+
+/* Bind `buf` to an empty cache. */
+DSA_API int idx_cache_init(dsa_index_cache* cache, int32_t* buf, int64_t rows, int topk);
+/* Record that F layer `layer` has (been enqueued to) write(n) the buffer. */
+DSA_API int idx_cache_put(dsa_index_cache* cache, int layer, const char* pattern);
+/* Device pointer of the indices layer `layer` must use: the buffer written
+ * by the most recent F layer at or before `layer` in `pattern`.
+ * DSA_ERR_INVALID_ARG if that F layer has not written it. */
+DSA_API int idx_cache_get(const dsa_index_cache* cache, int layer, const char* pattern,
+                  const int32_t** idx);
+
+/* ======================================================================
+ * sparse_attn_topk -- attention over each query's selected tokens.
+ *
+ * [Explainer] §稀疏注意力: each token attends only to its top-k history
+ * tokens; §IndexShare 的共享机制: S layers reuse the indices with their own
+ * attention weights, so every layer calls this with its own Q/K/V.
+ *     O[b,i,h] = sum_{j in I[b,i]} softmax_j(scale * Q[b,i,h].K[b,j,g(h)]) V[b,j,g(h)]
+ * g(h) = h / (Hq/Hkv).  Entries of idx equal to -1 are skipped; any other
+ * value outside [0, n_kv) is skipped and flagged (DSA_STATUS_BAD_INDEX).
+ *   Q   [B, n_q, Hq, d_qk]  bf16
+ *   K   [B, n_kv, Hkv, d_qk] bf16
+ *   V   [B, n_kv, Hkv, d_v]  bf16, or NULL for the latent form: one row per
+ *       token (Hkv == 1) is the key (all d_qk dims) and the value (its
+ *       first d_v dims).
+ *   idx [B, n_q, topk] int32
+ *   O   [B, n_q, Hq, d_v]   fp32 (o_dtype DSA_F32) or bf16 (DSA_BF16)
+ * Supported: d_qk == d_v in {64, 128} with Hq/Hkv in {1,2,4,8,16};
+ * latent d_qk = 576, d_v = 512, Hkv = 1.
+ * ====================================================================== */
+DSA_API int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, int d_qk, int d_v,
+                                    int topk, size_t* bytes);
+DSA_API int sparse_attn_topk(const void* Q, const void* K, const void* V, const int32_t* idx,
+                     int B, int n_q, int n_kv, int Hq, int Hkv, int d_qk, int d_v, int topk,
+                     float scale, void* O, int o_dtype,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ======================================================================
+ * layer_group_forward -- one layer group: F layers index, S layers reuse.
+ *
+ * [QbitAI] §IndexCache: few layers keep an indexer, compute the top-k and
+ * cache it, the rest skip it and reuse the most recent result with one
+ * extra branch in the inference code; §GLM-5.2 and [Explainer] §sharing:
+ * groups of four, the first layer computes.  `pattern` is a string over
+ * {F, S} of length n_layers starting with F (e.g. "FSSS", "FSSSFSSS").
+ * For each layer l in order: if pattern[l]=='F', idx_score_topk writes
+ * the cache buffer; then sparse_attn_topk runs with layer l's own Q/K/V
+ * and the cached indices.  S layers launch no indexer work.
+ * ====================================================================== */
+typedef struct dsa_group_shape {
+    int B, n_q, q_pos0, n_kv;
+    int H_I, d_I, idx_dtype;      /* indexer (DSA_BF16 or DSA_E4M3) */
+    int Hq, Hkv, d_qk, d_v;       /* attention                      */
+    int topk;
+    float scale;                  /* <= 0 selects 1/sqrt(d_qk)      */
+    int o_dtype;                  /* DSA_F32 or DSA_BF16            */
+} dsa_group_shape;
+
+typedef struct dsa_layer_args {
+    /* indexer inputs, read on F layers only (may be NULL on S layers) */
+    const void* q_I; const float* q_scale; const void* k_I; const float* k_scale; const float* w;
+    /* attention inputs and output of this layer */
+    const void* Q; const void* K; const void* V; void* O;
+} dsa_layer_args;
+
+typedef struct dsa_group_stats {
+    int indexer_launches;     /* idx_score_topk calls made           */
+    int attention_launches;   /* sparse_attn_topk calls made         */
+    /* Optional per-layer timing.  If non-NULL, `events` holds 3*n_layers
+     * cudaEvent_t handles (as void*) owned by the caller; on `stream` the
+     * library records events[3l] before layer l's indexer launch,
+     * events[3l+1] after it (same point on S layers) and events[3l+2]
+     * after layer l's attention launch. */
+    void* const* events;
+} dsa_group_stats;
+
+DSA_API int layer_group_forward_workspace_size(const dsa_group_shape* shape, size_t* bytes);
+DSA_API int layer_group_forward(const dsa_group_shape* shape, const dsa_layer_args* layers, int n_layers,
+                        const char* pattern, dsa_index_cache* cache, dsa_group_stats* stats,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H_ */
