@@ -240,6 +240,37 @@ DSA_API int layer_group_forward(const dsa_group_shape* shape, const dsa_layer_ar
                         const char* pattern, dsa_index_cache* cache, dsa_group_stats* stats,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* ======================================================================
+ * idx_score_topk_noalloc -- idx_score_topk for callers that cannot
+ * allocate device memory.  (The pages have no counterpart: this is a
+ * deployment variant of the same fused indexer + top-k.)
+ *
+ * Who needs it: code that runs inside another runtime's memory pool (an
+ * inference server or graph executor that owns every device allocation and
+ * forbids cudaMalloc, which can also synchronise the whole device), or a
+ * latency-critical path that must not allocate.  Such callers cannot
+ * provide the workspace idx_score_topk asks for.  This entry point takes
+ * only the inputs and the output (same meaning and layout as
+ * idx_score_topk) and keeps its scratch in one fixed 32 MiB array inside
+ * the library; it calls no allocator.
+ *   - The array is held by every GPU that loads the library until exit.
+ *   - The kernel's grid is capped to the CTAs whose top-k candidate buffers
+ *     fit in the array (63 at H_I = 32, topk = 2048), so big problems run
+ *     more slowly than with a full workspace.  A problem whose single CTA
+ *     needs more than the array is rejected with DSA_ERR_UNSUPPORTED.
+ *   - All calls share the array and it keeps the last call's contents;
+ *     each call clears the part that must start at zero.  Calls that
+ *     overlap on the GPU race on it and must be serialised by the caller.
+ *   - The first call on each device resolves the array's address
+ *     (cudaGetSymbolAddress); make that first call before any stream
+ *     capture begins.
+ *   - Device-side status (timeouts) is not reported by this entry point.
+ * ====================================================================== */
+DSA_API int idx_score_topk_noalloc(const void* q_I, const float* q_scale, const void* k_I,
+                                   const float* k_scale, const float* w, int dtype, int B, int n_q,
+                                   int q_pos0, int n_kv, int H_I, int d_I, int topk,
+                                   int32_t* idx_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

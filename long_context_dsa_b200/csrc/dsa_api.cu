@@ -105,6 +105,14 @@ int check_attn_shape(const void* V, int B, int n_q, int n_kv, int Hq, int Hkv, i
 
 }  // namespace
 
+namespace dsa {
+// Lets other translation units of the library report through dsa_last_error().
+int set_last_error(int code, const char* msg) {
+    g_last_error = msg ? msg : "";
+    return code;
+}
+}  // namespace dsa
+
 extern "C" {
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }

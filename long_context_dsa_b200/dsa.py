@@ -28,6 +28,7 @@ ABI_SYMBOLS = (
     "idx_cache_init", "idx_cache_put", "idx_cache_get",
     "sparse_attn_topk_workspace_size", "sparse_attn_topk",
     "layer_group_forward_workspace_size", "layer_group_forward",
+    "idx_score_topk_noalloc",
 )
 
 
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
         "layer_group_forward_workspace_size": ([ctypes.POINTER(GroupShape), psz], i),
         "layer_group_forward": ([ctypes.POINTER(GroupShape), ctypes.POINTER(LayerArgs), i, ctypes.c_char_p,
                                  ctypes.POINTER(IndexCacheStruct), ctypes.POINTER(GroupStats), vp, sz, vp], i),
+        "idx_score_topk_noalloc": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -312,3 +314,23 @@ def layer_group_forward(shape: GroupShape, layers, pattern: str, cache: IndexCac
     _check(lib().layer_group_forward(ctypes.byref(shape), arr, len(layers), pattern.encode(), ctypes.byref(cache.c),
                                      ctypes.byref(stats), _ptr(workspace), workspace.numel(), _stream(stream)))
     return stats
+
+
+# ------------------------------------------------- no-allocation variant
+def idx_score_topk_noalloc(q_I, k_I, w, topk: int, q_pos0: int = 0, q_scale=None, k_scale=None,
+                           out=None, stream=None) -> torch.Tensor:
+    """idx_score_topk without a workspace, for callers that cannot allocate device memory
+    (e.g. code running inside another runtime's memory pool).  Scratch lives in a fixed
+    32 MiB array inside the library; calls must not overlap on the GPU.  `out` should be
+    passed by such callers (allocating it here is only a convenience for tests)."""
+    dt = _idx_dtype(q_I)
+    B, n_q, H, d, n_kv = _idx_dims(q_I, k_I, q_pos0)
+    for t, n in ((q_I, "q_I"), (k_I, "k_I")):
+        _need(t, q_I.dtype, n)
+    _need(w, torch.float32, "w")
+    if out is None:
+        out = torch.empty((B, n_q, topk), dtype=torch.int32, device=q_I.device)
+    _need(out, torch.int32, "out")
+    _check(lib().idx_score_topk_noalloc(_ptr(q_I), _ptr(q_scale), _ptr(k_I), _ptr(k_scale), _ptr(w), dt, B, n_q,
+                                        q_pos0, n_kv, H, d, topk, _ptr(out), _stream(stream)))
+    return out
