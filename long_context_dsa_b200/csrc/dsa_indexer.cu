@@ -229,14 +229,16 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else {
         // ================================================== epilogue groups
-        const int g = warp >> 2;          // accumulator / query group
+        const int g = warp >> 2;            // accumulator / query group
         const int tid = threadIdx.x & 127;  // thread within the group == key lane
-        const int wq = warp & 3;          // TMEM lane quadrant
+        const int wq = warp & 3;            // TMEM lane quadrant
         TopkGroup<128> grp{tid, 1 + g, &sSc[g], p.cap};
         float* ws = sW + g * 256;
         TopkRowState* st = sSt + g * C::QG;
         int* sortbuf = sSort + g * DSA_TOPK_MAX;
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + g * 256;
+        constexpr int CHECK = 4;               // prune checks every CHECK key tiles
+        const int room = p.cap - CHECK * 128;  // prune a row once its buffer holds more than this
         uint32_t u = 0;
         bool ok = true;
         for (int r = 0; ok; ++r) {
@@ -262,6 +264,16 @@ __global__ void __launch_bounds__(320, 1)
             if (tid < C::QG) topk_row_init(&st[tid]);
             grp.sync();
             uint32_t* cbase = p.cand + (static_cast<size_t>(blockIdx.x) * 2 + g) * C::QG * 2 * p.cap;
+            // admission thresholds of this group's rows, in registers: admit a score iff it ranks
+            // above (thr_f, thr_i); they only ever trail the exact ones in shared memory, which
+            // admits a little more but never drops a true top-k entry
+            float thr_f[C::QG];
+            int thr_i[C::QG];
+#pragma unroll
+            for (int q = 0; q < C::QG; ++q) {
+                thr_f[q] = -INFINITY;
+                thr_i[q] = 0x7fffffff;
+            }
 
             for (int j = 0; j < nkt; ++j, ++u) {
                 const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[g], u & 1));
@@ -273,9 +285,12 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 } else {
                     tc::fence_after_sync();
-                    float sc[C::QG];
+                    // score[q] = sum_h w[q,h] * ReLU(acc[q,h]) with packed fp32x2 FMAs
+                    unsigned long long acc2[C::QG][H >= 32 ? 4 : 1];
 #pragma unroll
-                    for (int q = 0; q < C::QG; ++q) sc[q] = 0.f;
+                    for (int q = 0; q < C::QG; ++q)
+#pragma unroll
+                        for (int e = 0; e < (H >= 32 ? 4 : 1); ++e) acc2[q][e] = 0ull;
                     uint32_t va[32], vb[32];
                     tc::tmem_ld32(tbase, va);
                     tc::tmem_wait_ld_dep(va);
@@ -284,27 +299,41 @@ __global__ void __launch_bounds__(320, 1)
                         uint32_t(&cur)[32] = (c & 1) ? vb : va;
                         uint32_t(&nxt)[32] = (c & 1) ? va : vb;
                         if (c + 1 < 8) tc::tmem_ld32(tbase + (c + 1) * 32, nxt);
-                        float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
-                            const float4 wv = *reinterpret_cast<const float4*>(ws + c * 32 + i);
-                            const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+                        for (int i = 0; i < 16; i += 2) {
+                            const ulonglong2 w4 = *reinterpret_cast<const ulonglong2*>(ws + c * 32 + 2 * i);
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int col = c * 32 + i + e;
-                                const float x = fmaxf(__uint_as_float(cur[i + e]), 0.f);
-                                if (H >= 32) {
-                                    part[e] = fmaf(wa[e], x, part[e]);
-                                } else {
-                                    sc[col / H] = fmaf(wa[e], x, sc[col / H]);
-                                }
+                            for (int e = 0; e < 2; ++e) {
+                                const int pr = i + e;                 // column pair within the chunk
+                                const int q = (c * 32 + 2 * pr) / H;  // both columns of a pair share a query
+                                const unsigned long long x2 =
+                                    tc::pack2(fmaxf(__uint_as_float(cur[2 * pr]), 0.f),
+                                              fmaxf(__uint_as_float(cur[2 * pr + 1]), 0.f));
+                                const unsigned long long wv = e ? w4.y : w4.x;
+                                if (H >= 32)
+                                    tc::fma2(acc2[q][pr & 3], wv, x2);
+                                else
+                                    tc::fma2(acc2[q][0], wv, x2);
                             }
                         }
-                        if (H >= 32) sc[(c * 32) / H] += (part[0] + part[1]) + (part[2] + part[3]);
                         if (c + 1 < 8) tc::tmem_wait_ld_dep(nxt);
                     }
                     tc::fence_before_sync();
                     mbar_arrive(&acc_empty[g]);
+                    float sc[C::QG];
+#pragma unroll
+                    for (int q = 0; q < C::QG; ++q) {
+                        float2 t = tc::unpack2(acc2[q][0]);
+                        float sum = t.x + t.y;
+                        if (H >= 32) {
+#pragma unroll
+                            for (int e = 1; e < 4; ++e) {
+                                t = tc::unpack2(acc2[q][e]);
+                                sum += t.x + t.y;
+                            }
+                        }
+                        sc[q] = sum;
+                    }
 
                     const int s_key = j * 128 + tid;  // key position within the batch
                     if (FP8) {
@@ -320,31 +349,44 @@ __global__ void __launch_bounds__(320, 1)
                                 p.scores[(static_cast<size_t>(b) * p.n_q + qi) * p.n_kv + s_key] =
                                     (s_key <= p.q_pos0 + qi) ? sc[q] : -INFINITY;
                         }
-                    }
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < C::QG && !SCORES; ++q) {
-                        const int qi = qg0 + q;
-                        const bool valid = (qi < p.n_q) && (s_key <= p.q_pos0 + qi);
-                        const uint32_t key = score_key(sc[q]);
-                        const bool adm = valid && topk_admit(&st[q], key, s_key);
-                        uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
-                        topk_append_warp(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), key, s_key, adm, p.cap, p.hdr);
+                        for (int q = 0; q < C::QG; ++q) {
+                            const int qi = qg0 + q;
+                            const bool valid = (qi < p.n_q) && (s_key <= p.q_pos0 + qi);
+                            const bool adm = valid && (sc[q] > thr_f[q] || (sc[q] == thr_f[q] && s_key < thr_i[q]));
+                            if (__any_sync(0xffffffffu, adm)) {
+                                uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
+                                topk_append_warp(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), score_key(sc[q]),
+                                                 s_key, adm, p.cap, p.hdr);
+                            }
+                        }
                     }
                 }
-                grp.sync();
-                // decisions every thread of the group takes alike (read between two barriers)
-                unsigned long long need = 0ull;
+                if ((j % CHECK) == CHECK - 1 || j == nkt - 1) {
+                    grp.sync();
+                    // decisions every thread of the group takes alike (read between two barriers)
+                    unsigned long long need = 0ull;
 #pragma unroll
-                for (int q = 0; q < C::QG; ++q) need |= (st[q].count > p.cap - 128) ? (1ull << q) : 0ull;
-                const bool stop = wg_abort[g] != 0;
-                grp.sync();
-                if (stop) { ok = false; break; }
-                if (!SCORES && need) {
+                    for (int q = 0; q < C::QG; ++q)
+                        need |= (st[q].count > room && st[q].count > p.topk) ? (1ull << q) : 0ull;
+                    const bool stop = wg_abort[g] != 0;
+                    grp.sync();
+                    if (stop) { ok = false; break; }
+                    if (!SCORES && need) {
 #pragma unroll 1
-                    for (int q = 0; q < C::QG; ++q) {
-                        if ((need >> q) & 1ull) {
-                            uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
-                            grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk);
+                        for (int q = 0; q < C::QG; ++q) {
+                            if ((need >> q) & 1ull) {
+                                uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
+                                grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < C::QG; ++q) {
+                            if ((need >> q) & 1ull) {
+                                thr_f[q] = key_score(st[q].thr_key);
+                                thr_i[q] = st[q].thr_idx;
+                            }
                         }
                     }
                 }
@@ -403,9 +445,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, in
     return r == CUDA_SUCCESS;
 }
 
+// Candidate buffer entries per row: room for the k survivors of a prune plus at
+// least 4 tiles of appends (the epilogue checks every 4 key tiles) and slack.
 int cand_cap(int topk) {
     int c = 2 * topk + 256;
-    if (c < 512) c = 512;
+    if (c < topk + 4 * 128 + 512) c = topk + 4 * 128 + 512;
     if (c > kCandCap) c = kCandCap;
     return c;
 }

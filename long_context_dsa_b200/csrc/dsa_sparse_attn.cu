@@ -4,27 +4,31 @@
 // history tokens; §IndexShare 的共享机制: S layers keep their own attention
 // weights, so each layer runs this kernel with its own Q/K/V.
 //
-// Design (B200): the work is a gather -- every query reads k rows of K and
-// V picked by the index cache -- so it is bound by HBM, not by math.
-//   * A persistent CTA owns (query row, block of HB KV heads) items.  One
-//     producer warp streams the selected rows into a multi-stage shared
-//     memory ring with one bulk async copy (cp.async.bulk, TMA engine) per
-//     gathered row: a row of HB*D bf16 is contiguous in the token-major
-//     K/V layout.  Completion is tracked by mbarrier transaction bytes.
-//   * HB consumer warps, one per KV head, run an online-softmax attention
-//     over the chunk with warp-level bf16 tensor-core MMAs (m16n8k16):
-//     S^T = K_chunk Q^T puts keys on M and the GQA group's query heads on
-//     N (8 columns, no padding at G = 8); O^T += V^T P uses d on M.  The
-//     probabilities move from the S^T accumulator layout into the B
-//     operand layout with movmatrix.  P is split into bf16 hi + lo parts
-//     (two MMAs) so the weights keep ~16 bits of precision.
-//   * Rows are stored at a stride of RB+16 bytes, which makes every
-//     ldmatrix conflict-free without swizzling the copies.
+// Design (B200): the work is a gather -- every (query, KV head) reads k
+// rows of K and V picked by the index cache -- so it is bound by memory,
+// not by math.
+//   * The unit of work is one (query row, KV head).  Every warp runs its own
+//     pipeline over units: it gathers its head's K and V slices (d bf16
+//     each, contiguous in the token-major layout) for a chunk of selected
+//     tokens with 16-byte cp.async into a private multi-stage ring, and
+//     computes on the oldest stage while the younger ones are in flight.
+//     Padding entries (-1) become zero-filled copies that read nothing.
+//     The next chunk's indices are loaded one iteration ahead, so neither
+//     the index load nor a shared producer sits on the critical path.
+//   * Online softmax with warp-level bf16 tensor-core MMAs (m16n8k16):
+//     S^T = K_chunk Q^T puts keys on M and the GQA group's query heads on N
+//     (8 columns: no padding at G = 8); O^T += V^T P puts d on M.  P moves
+//     from the S^T accumulator layout into the B-operand layout with
+//     movmatrix and is split into bf16 hi + lo parts (two MMAs) so the
+//     weights keep ~16 bits.
+//   * Ring rows are packed at 2*d bytes with their 16-byte segments XOR-
+//     swizzled by (row & 7): every ldmatrix is conflict-free and 14 warps
+//     (16-key chunks, 2 stages each) fit in shared memory at d = 128.  On
+//     B200 the number of warps in flight set the speed far more than the
+//     stages per warp did.
 #include "dsa_common.cuh"
 
 namespace dsa {
-
-static constexpr int kAttnChunk = 32;  // gathered keys per pipeline stage
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -53,115 +57,98 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
+// 16-byte async copy global -> shared; src_bytes = 0 writes zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-template <int D, int HB, int STAGES>
+// SWZ: rows packed at 2*d bytes with their 16-byte segments XOR-swizzled by
+// (row & 7) instead of padded, which fits more warps in shared memory.
+template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ = false>
 struct AttnCfg {
-    static constexpr int RB = HB * D * 2;         // bytes of one gathered row (HB heads)
-    static constexpr int RS = RB + 16;            // smem row stride (bank-conflict free)
-    static constexpr int STAGE_BYTES = 2 * kAttnChunk * RS;
-    static constexpr int THREADS = (HB + 1) * 32;
-    static constexpr size_t SMEM = static_cast<size_t>(STAGES) * STAGE_BYTES + STAGES * kAttnChunk * 4 +
-                                   2 * STAGES * 8 + 16;
+    static constexpr int RS = SWZ ? D * 2 : D * 2 + 16;    // ring row stride (bytes)
+    static constexpr int STAGE_BYTES = 2 * CHUNK * RS;     // K rows then V rows
+    static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + STAGES * CHUNK * 4;  // + staged indices
+    static constexpr int SEGS = D * 2 / 16;                // 16-byte segments per row slice
+    static constexpr int KEYS_PER_INSN = 32 / SEGS;        // rows one warp-wide cp.async covers
+    static constexpr size_t SMEM = static_cast<size_t>(WARPS) * WARP_BYTES;
+    static_assert(CHUNK % 16 == 0 && CHUNK <= 32, "chunk of whole 16-key MMA tiles, one index per lane");
+    static_assert(32 % SEGS == 0, "row slice splits evenly over the warp");
+    // byte offset of 16-byte segment `sg` of ring row `r`
+    __device__ static __forceinline__ uint32_t at(int r, int sg) {
+        return static_cast<uint32_t>(r * RS + ((SWZ ? (sg ^ (r & 7)) : sg) << 4));
+    }
 };
 
-template <int D, int HB, int STAGES, bool OUT_BF16>
-__global__ void __launch_bounds__(AttnCfg<D, HB, STAGES>::THREADS, 1)
+template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ, bool QK_SPLIT, bool OUT_BF16>
+__global__ void __launch_bounds__(WARPS * 32)
     sparse_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                        const __nv_bfloat16* __restrict__ V, const int* __restrict__ idx, int B, int n_q,
                        int n_kv, int Hq, int Hkv, int topk, float scale_log2, void* __restrict__ O,
                        WsHeader* hdr) {
-    using C = AttnCfg<D, HB, STAGES>;
+    using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char* stage_base = smem;
-    int* sidx = reinterpret_cast<int*>(smem + STAGES * C::STAGE_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(sidx + STAGES * kAttnChunk);
-    uint64_t* empty = full + STAGES;
-    int* abort_flag = reinterpret_cast<int*>(empty + STAGES);
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char* ring = smem + warp * C::WARP_BYTES;
+    int* sidx = reinterpret_cast<int*>(ring + STAGES * C::STAGE_BYTES);
+    const uint32_t ring_s = smem_u32(ring);
+
     const int G = Hq / Hkv;
-    const int hblocks = Hkv / HB;
-    const long long total = static_cast<long long>(B) * n_q * hblocks;
-    const int nchunks = (topk + kAttnChunk - 1) / kAttnChunk;
+    const long long units = static_cast<long long>(B) * n_q * Hkv;
+    const int nchunks = (topk + CHUNK - 1) / CHUNK;
+    const size_t tok_stride = static_cast<size_t>(Hkv) * D;  // elements per token row of K / V
 
-    // zero the ring once: rows never written by a copy must hold finite data
-    for (int i = threadIdx.x; i < STAGES * C::STAGE_BYTES / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(stage_base)[i] = make_uint4(0, 0, 0, 0);
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], HB);
-        }
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-
-    if (warp == HB) {
-        // ------------------------------------------------------------ producer
-        int last_round[STAGES];
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
-        long long it = 0;
-        bool ok_run = true;
-        for (long long w = blockIdx.x; w < total && ok_run; w += gridDim.x) {
-            const long long row = w / hblocks;
-            const int hb = static_cast<int>(w % hblocks);
-            const long long b = row / n_q;
-            const int* irow = idx + row * topk;
-            const size_t tok_stride = static_cast<size_t>(Hkv) * D;  // elements per token
-            const __nv_bfloat16* kb = K + static_cast<size_t>(b) * n_kv * tok_stride + static_cast<size_t>(hb) * HB * D;
-            const __nv_bfloat16* vb = V + static_cast<size_t>(b) * n_kv * tok_stride + static_cast<size_t>(hb) * HB * D;
-            for (int c = 0; c < nchunks; ++c, ++it) {
-                const int s = static_cast<int>(it % STAGES);
-                const int r = static_cast<int>(it / STAGES);
-                if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1)) {
-                    if (lane == 0) raise_status(hdr, DSA_STATUS_TIMEOUT, 0x5a01);
-                    ok_run = false;
-                    break;
-                }
-                const int kk = c * kAttnChunk + lane;
-                const int t = (kk < topk) ? __ldg(irow + kk) : -1;
-                const bool ok = (t >= 0) && (t < n_kv);
-                if (t < -1 || t >= n_kv) raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
-                sidx[s * kAttnChunk + lane] = ok ? t : -1;
-                const unsigned m = __ballot_sync(0xffffffffu, ok);
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(m)) * 2u * C::RB);
-                __syncwarp();
-                if (ok) {
-                    unsigned char* krow = stage_base + s * C::STAGE_BYTES + lane * C::RS;
-                    unsigned char* vrow = krow + kAttnChunk * C::RS;
-                    bulk_g2s(krow, kb + static_cast<size_t>(t) * tok_stride, C::RB, &full[s]);
-                    bulk_g2s(vrow, vb + static_cast<size_t>(t) * tok_stride, C::RB, &full[s]);
-                }
-                last_round[s] = r;
-            }
-            if (__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(abort_flag) != 0)) break;
-        }
-        if (!ok_run && lane == 0) atomicExch(abort_flag, 1);
-        // never leave with copies in flight into this CTA's shared memory
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s)
-            if (last_round[s] >= 0 && !mbar_wait(&full[s], last_round[s] & 1) && lane == 0)
-                raise_status(hdr, DSA_STATUS_TIMEOUT, 0x5a02);
-        return;
-    }
-
-    // ---------------------------------------------------------------- consumers
-    const int cw = warp;  // KV head within the block
-    const int qn = lane >> 2;          // query head (N column) this lane loads for Q
-    const int hc = 2 * (lane & 3);     // first of the two head columns this lane owns in C tiles
+    const int qn = lane >> 2;        // query head (N column) this lane loads for Q; key row in C tiles
+    const int hc = 2 * (lane & 3);   // first of the two head columns this lane owns in C tiles
     const int lrow = lane & 7, lq = lane >> 3;
-    // ldmatrix lane offsets
     const int k_key_off = ((lq & 1) ? 8 : 0) + lrow, k_d_off = (lq >= 2) ? 8 : 0;   // K: non-trans A
     const int v_key_off = ((lq >= 2) ? 8 : 0) + lrow, v_d_off = (lq & 1) ? 8 : 0;  // V: trans A
-    long long it = 0;
-    for (long long w = blockIdx.x; w < total; w += gridDim.x) {
-        const long long row = w / hblocks;
-        const int hb = static_cast<int>(w % hblocks);
-        const int g = hb * HB + cw;  // KV head
+    const int seg = lane % C::SEGS, sub = lane / C::SEGS;  // copy: segment within a row, row within an insn
+
+    for (long long u = static_cast<long long>(blockIdx.x) * WARPS + warp; u < units;
+         u += static_cast<long long>(gridDim.x) * WARPS) {
+        const long long row = u / Hkv;
+        const int g = static_cast<int>(u % Hkv);
+        const long long b = row / n_q;
+        const int* irow = idx + row * topk;
+        const __nv_bfloat16* kb = K + static_cast<size_t>(b) * n_kv * tok_stride + static_cast<size_t>(g) * D;
+        const __nv_bfloat16* vb = V + static_cast<size_t>(b) * n_kv * tok_stride + static_cast<size_t>(g) * D;
+
+        // index of key `lane` of chunk c (-1 past the end); out-of-range entries are flagged and skipped
+        auto load_idx = [&](int c) -> int {
+            const int kk = c * CHUNK + lane;
+            int t = (lane < CHUNK && kk < topk) ? __ldg(irow + kk) : -1;
+            if (t < -1 || t >= n_kv) {
+                raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
+                t = -1;
+            }
+            return t;
+        };
+        // gather chunk c's K and V slices into stage c % STAGES (always commits one group)
+        auto issue = [&](int c, int tsel) {
+            if (c < nchunks) {
+                const int s = c % STAGES;
+                if (lane < CHUNK) sidx[s * CHUNK + lane] = tsel;
+                const uint32_t kst = ring_s + s * C::STAGE_BYTES;
+                const uint32_t vst = kst + CHUNK * C::RS;
+#pragma unroll
+                for (int i = 0; i < CHUNK / C::KEYS_PER_INSN; ++i) {
+                    const int key = i * C::KEYS_PER_INSN + sub;
+                    const int t = __shfl_sync(0xffffffffu, tsel, key);
+                    const uint32_t nb = t >= 0 ? 16u : 0u;
+                    const size_t off = static_cast<size_t>(t >= 0 ? t : 0) * tok_stride + seg * 8;
+                    cp_async16(kst + C::at(key, seg), kb + off, nb);
+                    cp_async16(vst + C::at(key, seg), vb + off, nb);
+                }
+            }
+            cp_async_commit();
+        };
+
         // Q^T fragments: B[k=d][n=head]
         uint32_t qf[D / 16][2];
         {
@@ -178,39 +165,47 @@ __global__ void __launch_bounds__(AttnCfg<D, HB, STAGES>::THREADS, 1)
         for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
         float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
 
-        bool alive = true;
-        for (int c = 0; c < nchunks; ++c, ++it) {
-            const int s = static_cast<int>(it % STAGES);
-            const int r = static_cast<int>(it / STAGES);
-            if (!mbar_wait(&full[s], r & 1)) {
-                if (lane == 0) {
-                    raise_status(hdr, DSA_STATUS_TIMEOUT, 0x5a03);
-                    atomicExch(abort_flag, 1);
-                }
-                alive = false;
-                break;
-            }
-            const unsigned char* kst = stage_base + s * C::STAGE_BYTES;
-            const unsigned char* vst = kst + kAttnChunk * C::RS;
-            const int* si = sidx + s * kAttnChunk;
-            // ---- S^T = K Q^T  (two 16-key tiles)
-            float sacc[2][4];
+        // prologue: stages 0 .. STAGES-2 in flight, the next chunk's indices in a register
+        __syncwarp();
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+        for (int c = 0; c < STAGES - 1; ++c) issue(c, load_idx(c));
+        int t_next = load_idx(STAGES - 1);
+
+        for (int c = 0; c < nchunks; ++c) {
+            issue(c + STAGES - 1, t_next);
+            t_next = load_idx(c + STAGES);
+            cp_async_wait<STAGES - 1>();
+            __syncwarp();
+            const int s = c % STAGES;
+            const uint32_t kst = ring_s + s * C::STAGE_BYTES;
+            const uint32_t vst = kst + CHUNK * C::RS;
+            const int* si = sidx + s * CHUNK;
+            constexpr int MT = CHUNK / 16;
+            // ---- S^T = K Q^T
+            float sacc[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                float s2[4] = {0.f, 0.f, 0.f, 0.f};  // second accumulation chain (QK_SPLIT)
                 sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
-                const uint32_t abase =
-                    smem_u32(kst + (mt * 16 + k_key_off) * C::RS + (cw * D + k_d_off) * 2);
+                const int krow = mt * 16 + k_key_off;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4(abase + ks * 32, a0, a1, a2, a3);
-                    mma_bf16(sacc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                    ldsm_x4(kst + C::at(krow, 2 * ks + k_d_off / 8), a0, a1, a2, a3);
+                    if (QK_SPLIT && (ks & 1))
+                        mma_bf16(s2, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                    else
+                        mma_bf16(sacc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                }
+                if (QK_SPLIT) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sacc[mt][e] += s2[e];
                 }
             }
             // ---- mask, scale, online softmax
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < MT; ++mt) {
                 const bool v0 = si[mt * 16 + qn] >= 0;
                 const bool v1 = si[mt * 16 + qn + 8] >= 0;
 #pragma unroll
@@ -233,9 +228,9 @@ __global__ void __launch_bounds__(AttnCfg<D, HB, STAGES>::THREADS, 1)
                 mrun[j] = mnew[j];
                 lrun[j] *= alpha[j];
             }
-            uint32_t phi[2][2], plo[2][2];  // [k-step][matrix rows 0-7 / 8-15]
+            uint32_t phi[MT][2], plo[MT][2];  // [k-step][key rows 0-7 / 8-15]
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < MT; ++mt) {
                 float p[4];
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
@@ -262,18 +257,16 @@ __global__ void __launch_bounds__(AttnCfg<D, HB, STAGES>::THREADS, 1)
                 o[dt][2] *= alpha[0];
                 o[dt][3] *= alpha[1];
 #pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
+                for (int ks = 0; ks < MT; ++ks) {
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(smem_u32(vst + (ks * 16 + v_key_off) * C::RS + (cw * D + dt * 16 + v_d_off) * 2), a0,
-                              a1, a2, a3);
+                    ldsm_x4_t(vst + C::at(ks * 16 + v_key_off, 2 * dt + v_d_off / 8), a0, a1, a2, a3);
                     mma_bf16(o[dt], a0, a1, a2, a3, phi[ks][0], phi[ks][1]);
                     mma_bf16(o[dt], a0, a1, a2, a3, plo[ks][0], plo[ks][1]);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            __syncwarp();  // every lane is done with stage s before it is refilled
         }
-        if (!alive) break;
+        cp_async_wait<0>();  // retire the trailing (empty) groups before the ring is reused
         // ---- finalize: row sums across the 8 lanes sharing a head column
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -303,26 +296,31 @@ __global__ void __launch_bounds__(AttnCfg<D, HB, STAGES>::THREADS, 1)
                 }
             }
         }
-        if (*reinterpret_cast<volatile int*>(abort_flag) != 0) break;
     }
 }
 
-template <int D, int HB, int STAGES>
+template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ = false, bool QK_SPLIT = false>
 static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                                  const int* idx, int B, int n_q, int n_kv, int Hq, int Hkv, int topk,
                                  float scale, void* O, bool out_bf16, WsHeader* hdr, int num_sms,
                                  cudaStream_t stream) {
-    using C = AttnCfg<D, HB, STAGES>;
-    auto kern = out_bf16 ? sparse_attn_kernel<D, HB, STAGES, true> : sparse_attn_kernel<D, HB, STAGES, false>;
+    using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
+    auto kern = out_bf16 ? sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, true>
+                         : sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
     if (e != cudaSuccess) return e;
-    const long long total = static_cast<long long>(B) * n_q * (Hkv / HB);
-    long long grid = num_sms;
-    if (grid > total) grid = total;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, C::SMEM);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const long long units = static_cast<long long>(B) * n_q * Hkv;
+    long long grid = static_cast<long long>(num_sms) * per_sm;
+    const long long need = (units + WARPS - 1) / WARPS;
+    if (grid > need) grid = need;
     if (grid < 1) grid = 1;
     const float scale_log2 = scale * 1.4426950408889634f;
-    kern<<<static_cast<int>(grid), C::THREADS, C::SMEM, stream>>>(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, topk,
-                                                                  scale_log2, O, hdr);
+    kern<<<static_cast<int>(grid), WARPS * 32, C::SMEM, stream>>>(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, topk,
+                                                                   scale_log2, O, hdr);
     return cudaGetLastError();
 }
 
@@ -333,20 +331,14 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
     auto q = static_cast<const __nv_bfloat16*>(Q);
     auto k = static_cast<const __nv_bfloat16*>(K);
     auto v = static_cast<const __nv_bfloat16*>(V);
-    if (d == 128) {
-        if (Hkv % 4 == 0)
-            return launch_attn_t<128, 4, 3>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, hdr, num_sms, stream);
-        if (Hkv % 2 == 0)
-            return launch_attn_t<128, 2, 4>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, hdr, num_sms, stream);
-        return launch_attn_t<128, 1, 6>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, hdr, num_sms, stream);
-    }
-    if (d == 64) {
-        if (Hkv % 8 == 0)
-            return launch_attn_t<64, 8, 3>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, hdr, num_sms, stream);
-        if (Hkv % 4 == 0)
-            return launch_attn_t<64, 4, 4>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, hdr, num_sms, stream);
-        return launch_attn_t<64, 1, 6>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, hdr, num_sms, stream);
-    }
+    // 16-key chunks, 2 stages per warp, swizzled rows: as many warps per SM as shared memory
+    // holds (measured on B200: warps in flight matter more than stages per warp).
+    if (d == 128)
+        return launch_attn_t<128, 16, 2, 14, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
+                                                         out_bf16, hdr, num_sms, stream);
+    if (d == 64)
+        return launch_attn_t<64, 16, 2, 16, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
+                                                        out_bf16, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }
 

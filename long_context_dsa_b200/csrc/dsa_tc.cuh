@@ -63,6 +63,22 @@ __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
         : "memory");
 }
 
+// ------------------------------------------------------- packed fp32 pairs
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 unpack2(unsigned long long r) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
+    return f;
+}
+// acc.{x,y} = a.{x,y} * b.{x,y} + acc.{x,y}, both lanes rounded to nearest (sm_100 packed FMA)
+__device__ __forceinline__ void fma2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
 // ------------------------------------------------------------------- MMA
 // D[tmem] (+)= A[smem] * B[smem]^T, one CTA, issued by one thread.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {

@@ -180,6 +180,7 @@ struct TopkGroup {
     // All NT threads call it; st->count is read after a group barrier.
     __device__ void prune(TopkRowState* st, uint32_t* ckey, int* cidx, int k) const {
         const int n = min(st->count, cap);
+        if (n <= k) return;  // nothing to drop (every thread reads the same n)
         uint32_t rk[PER];
         int ri[PER];
         uint32_t valid = 0u;

@@ -28,6 +28,10 @@ CASES = [
     ("decode_b3", 3, 1, 2999, 3000, 32, 128, 512, dict(r=32, base_std=1.0, noise_std=0.2)),
     ("h16_777", 1, 777, 0, 777, 16, 128, 100, dict(r=32, base_std=1.0, noise_std=0.2)),
     ("h8_640", 1, 640, 0, 640, 8, 128, 64, dict(r=32, base_std=1.0, noise_std=0.2)),
+    # small top-k over many key tiles: frequent prunes, rows shorter than k at the start
+    ("h32_k16", 1, 1500, 0, 1500, 32, 128, 16, dict(r=32, base_std=1.0, noise_std=0.2)),
+    ("h64_k1", 1, 600, 0, 600, 64, 128, 1, dict(r=32, base_std=1.0, noise_std=0.2)),
+    ("h4_k3_b2", 2, 700, 0, 700, 4, 64, 3, dict(r=8, base_std=1 / 8, noise_std=1 / 8)),
 ]
 
 
