@@ -89,14 +89,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended up to `hint_ns` while
+// the phase is incomplete (fewer spin iterations stealing issue slots).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; false on timeout
 // (the caller then records DSA_STATUS_TIMEOUT and winds down).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+        if ((it & 15u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
     }
 }
 
@@ -118,9 +132,10 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
 // -0.0 and +0.0 map to the same key.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t score_key(float f) {
-    uint32_t u = __float_as_uint(f);
-    if (u == 0x80000000u) u = 0u;
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    // f + 0.0f turns -0.0 into +0.0 (round to nearest) and leaves every other value alone;
+    // then negative floats are bit-inverted and non-negative ones get the sign bit set
+    const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
+    return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ float key_score(uint32_t k) {

@@ -53,7 +53,7 @@ struct IdxCfg {
     static constexpr int OFF_W = OFF_A + STAGES * A_STAGE;
     static constexpr int OFF_ST = OFF_W + 2 * 256 * 4;
     static constexpr int OFF_SC = OFF_ST + 2 * QG * static_cast<int>(sizeof(TopkRowState));
-    static constexpr int OFF_SORT = OFF_SC + 2 * static_cast<int>(sizeof(TopkScratch));
+    static constexpr int OFF_SORT = OFF_SC + 2 * static_cast<int>(sizeof(TopkGroup<128>::Scratch));
     static constexpr int OFF_BAR = OFF_SORT + 2 * DSA_TOPK_MAX * 4;
     static constexpr int NBAR = 2 + 2 * STAGES + 4;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -86,12 +86,14 @@ __global__ void __launch_bounds__(320, 1)
                         const IdxParams p) {
     using C = IdxCfg<H, D, FP8>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte alignment for the swizzled operand tiles, by offsetting the shared array itself
+    // (an integer round trip would make every later access a generic one)
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     unsigned char* sB = smem + C::OFF_B;
     unsigned char* sA = smem + C::OFF_A;
     float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
     TopkRowState* sSt = reinterpret_cast<TopkRowState*>(smem + C::OFF_ST);
-    TopkScratch* sSc = reinterpret_cast<TopkScratch*>(smem + C::OFF_SC);
+    auto* sSc = reinterpret_cast<TopkGroup<128>::Scratch*>(smem + C::OFF_SC);
     int* sSort = reinterpret_cast<int*>(smem + C::OFF_SORT);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars + 0;
@@ -237,8 +239,9 @@ __global__ void __launch_bounds__(320, 1)
         TopkRowState* st = sSt + g * C::QG;
         int* sortbuf = sSort + g * DSA_TOPK_MAX;
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + g * 256;
-        constexpr int CHECK = 4;               // prune checks every CHECK key tiles
-        const int room = p.cap - CHECK * 128;  // prune a row once its buffer holds more than this
+        constexpr int CHECK = 4;                       // prune checks every CHECK key tiles
+        const int sub = grp.sub();                     // this warp's share of a row buffer
+        const int room = sub - CHECK * 32;             // prune once a sub-buffer holds more than this
         uint32_t u = 0;
         bool ok = true;
         for (int r = 0; ok; ++r) {
@@ -264,16 +267,15 @@ __global__ void __launch_bounds__(320, 1)
             if (tid < C::QG) topk_row_init(&st[tid]);
             grp.sync();
             uint32_t* cbase = p.cand + (static_cast<size_t>(blockIdx.x) * 2 + g) * C::QG * 2 * p.cap;
-            // admission thresholds of this group's rows, in registers: admit a score iff it ranks
-            // above (thr_f, thr_i); they only ever trail the exact ones in shared memory, which
-            // admits a little more but never drops a true top-k entry
-            float thr_f[C::QG];
-            int thr_i[C::QG];
+            uint32_t* wkey = cbase + wq * sub;                              // row 0, this warp's keys
+            int* widx = reinterpret_cast<int*>(cbase + p.cap) + wq * sub;  // row 0, this warp's indices
+            const int rstride = 2 * p.cap;                                  // 32-bit words per row
+            int cnt[C::QG];  // this warp's sub-buffer counts (warp-uniform; published at checks)
 #pragma unroll
-            for (int q = 0; q < C::QG; ++q) {
-                thr_f[q] = -INFINITY;
-                thr_i[q] = 0x7fffffff;
-            }
+            for (int q = 0; q < C::QG; ++q) cnt[q] = 0;
+            // rows of this group that exist, and the last key each may see
+            const int qlast = min(C::QG, p.n_q - qg0);
+            const int pos0 = p.q_pos0 + qg0;
 
             for (int j = 0; j < nkt; ++j, ++u) {
                 const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[g], u & 1));
@@ -285,12 +287,12 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 } else {
                     tc::fence_after_sync();
-                    // score[q] = sum_h w[q,h] * ReLU(acc[q,h]) with packed fp32x2 FMAs
-                    unsigned long long acc2[C::QG][H >= 32 ? 4 : 1];
+                    // score[q] = sum_h w[q,h] * ReLU(acc[q,h]) with packed fp32x2 FMAs; each
+                    // 32-column chunk holds whole queries' heads (H >= 32: part of one query;
+                    // H < 32: 32/H queries), so it is folded into sc[] as soon as it is done
+                    float sc[C::QG];
 #pragma unroll
-                    for (int q = 0; q < C::QG; ++q)
-#pragma unroll
-                        for (int e = 0; e < (H >= 32 ? 4 : 1); ++e) acc2[q][e] = 0ull;
+                    for (int q = 0; q < C::QG; ++q) sc[q] = 0.f;
                     uint32_t va[32], vb[32];
                     tc::tmem_ld32(tbase, va);
                     tc::tmem_wait_ld_dep(va);
@@ -299,41 +301,36 @@ __global__ void __launch_bounds__(320, 1)
                         uint32_t(&cur)[32] = (c & 1) ? vb : va;
                         uint32_t(&nxt)[32] = (c & 1) ? va : vb;
                         if (c + 1 < 8) tc::tmem_ld32(tbase + (c + 1) * 32, nxt);
+                        constexpr int NA = H >= 32 ? 4 : 32 / H;  // accumulators per chunk
+                        unsigned long long a2[NA];
+#pragma unroll
+                        for (int e = 0; e < NA; ++e) a2[e] = 0ull;
 #pragma unroll
                         for (int i = 0; i < 16; i += 2) {
                             const ulonglong2 w4 = *reinterpret_cast<const ulonglong2*>(ws + c * 32 + 2 * i);
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const int pr = i + e;                 // column pair within the chunk
-                                const int q = (c * 32 + 2 * pr) / H;  // both columns of a pair share a query
+                                const int pr = i + e;  // column pair within the chunk
                                 const unsigned long long x2 =
                                     tc::pack2(fmaxf(__uint_as_float(cur[2 * pr]), 0.f),
                                               fmaxf(__uint_as_float(cur[2 * pr + 1]), 0.f));
-                                const unsigned long long wv = e ? w4.y : w4.x;
-                                if (H >= 32)
-                                    tc::fma2(acc2[q][pr & 3], wv, x2);
-                                else
-                                    tc::fma2(acc2[q][0], wv, x2);
+                                tc::fma2(a2[H >= 32 ? (pr & 3) : (2 * pr) / H], e ? w4.y : w4.x, x2);
+                            }
+                        }
+                        if (H >= 32) {
+                            const float2 t = tc::unpack2(tc::add2(tc::add2(a2[0], a2[1 % NA]), tc::add2(a2[2 % NA], a2[3 % NA])));
+                            sc[(c * 32) / H] += t.x + t.y;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < NA; ++e) {
+                                const float2 t = tc::unpack2(a2[e]);
+                                sc[c * NA + e] = t.x + t.y;
                             }
                         }
                         if (c + 1 < 8) tc::tmem_wait_ld_dep(nxt);
                     }
                     tc::fence_before_sync();
                     mbar_arrive(&acc_empty[g]);
-                    float sc[C::QG];
-#pragma unroll
-                    for (int q = 0; q < C::QG; ++q) {
-                        float2 t = tc::unpack2(acc2[q][0]);
-                        float sum = t.x + t.y;
-                        if (H >= 32) {
-#pragma unroll
-                            for (int e = 1; e < 4; ++e) {
-                                t = tc::unpack2(acc2[q][e]);
-                                sum += t.x + t.y;
-                            }
-                        }
-                        sc[q] = sum;
-                    }
 
                     const int s_key = j * 128 + tid;  // key position within the batch
                     if (FP8) {
@@ -350,26 +347,38 @@ __global__ void __launch_bounds__(320, 1)
                                     (s_key <= p.q_pos0 + qi) ? sc[q] : -INFINITY;
                         }
                     } else {
+                        // every row sees every key of this tile unless the tile reaches the diagonal
+                        const bool full_tile = (j * 128 + 127 <= pos0) && (qlast == C::QG);
 #pragma unroll
                         for (int q = 0; q < C::QG; ++q) {
-                            const int qi = qg0 + q;
-                            const bool valid = (qi < p.n_q) && (s_key <= p.q_pos0 + qi);
-                            const bool adm = valid && (sc[q] > thr_f[q] || (sc[q] == thr_f[q] && s_key < thr_i[q]));
-                            if (__any_sync(0xffffffffu, adm)) {
-                                uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
-                                topk_append_warp(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), score_key(sc[q]),
-                                                 s_key, adm, p.cap, p.hdr);
-                            }
+                            const bool valid = full_tile | ((q < qlast) & (s_key <= pos0 + q));
+                            // admit iff the score ranks above the row's k-th candidate (set by the last prune)
+                            const uint32_t key = score_key(sc[q]);
+                            const uint32_t tk = st[q].thr_key;
+                            const bool adm = valid & ((key > tk) | ((key == tk) & (s_key < st[q].thr_idx)));
+                            topk_append_warp(wkey + q * rstride, widx + q * rstride, cnt[q], key, s_key, adm, sub);
                         }
                     }
                 }
                 if ((j % CHECK) == CHECK - 1 || j == nkt - 1) {
+                    if (lane == 0) {
+#pragma unroll
+                        for (int q = 0; q < C::QG; ++q) st[q].cnt[wq] = cnt[q];
+                    }
                     grp.sync();
                     // decisions every thread of the group takes alike (read between two barriers)
                     unsigned long long need = 0ull;
 #pragma unroll
-                    for (int q = 0; q < C::QG; ++q)
-                        need |= (st[q].count > room && st[q].count > p.topk) ? (1ull << q) : 0ull;
+                    for (int q = 0; q < C::QG; ++q) {
+                        int mx = 0, tot = 0;
+#pragma unroll
+                        for (int ww = 0; ww < 4; ++ww) {
+                            mx = max(mx, st[q].cnt[ww]);
+                            tot += st[q].cnt[ww];
+                        }
+                        need |= (mx > room && tot > p.topk) ? (1ull << q) : 0ull;
+                        if (mx > sub && tid == 0) raise_status(p.hdr, DSA_STATUS_OVERFLOW, mx);
+                    }
                     const bool stop = wg_abort[g] != 0;
                     grp.sync();
                     if (stop) { ok = false; break; }
@@ -378,16 +387,13 @@ __global__ void __launch_bounds__(320, 1)
                         for (int q = 0; q < C::QG; ++q) {
                             if ((need >> q) & 1ull) {
                                 uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
-                                grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk);
+                                grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk, room - 32);
                             }
                         }
 #pragma unroll
-                        for (int q = 0; q < C::QG; ++q) {
-                            if ((need >> q) & 1ull) {
-                                thr_f[q] = key_score(st[q].thr_key);
-                                thr_i[q] = st[q].thr_idx;
-                            }
-                        }
+                        for (int q = 0; q < C::QG; ++q)
+                            if ((need >> q) & 1ull) cnt[q] = st[q].cnt[wq];
+
                     }
                 }
             }
@@ -450,6 +456,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, in
 int cand_cap(int topk) {
     int c = 2 * topk + 256;
     if (c < topk + 4 * 128 + 512) c = topk + 4 * 128 + 512;
+    c = (c + 127) / 128 * 128;
     if (c > kCandCap) c = kCandCap;
     return c;
 }

@@ -74,6 +74,12 @@ __device__ __forceinline__ float2 unpack2(unsigned long long r) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
     return f;
 }
+// a.{x,y} + b.{x,y}, both lanes rounded to nearest (sm_100 packed add)
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 // acc.{x,y} = a.{x,y} * b.{x,y} + acc.{x,y}, both lanes rounded to nearest (sm_100 packed FMA)
 __device__ __forceinline__ void fma2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
     asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));

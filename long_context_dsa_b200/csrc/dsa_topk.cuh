@@ -5,107 +5,167 @@
 // top-k"): the k largest scores of the row, ties to the lower token index,
 // -0.0 equal to +0.0; output ascending by token index, then -1.
 //
-// A row's state is a candidate buffer of (key, index) pairs plus an
-// admission threshold.  Scores arrive in any order; an arriving pair is
-// kept iff it ranks above the current k-th candidate.  When the buffer
-// nears its capacity the group of NT threads that owns the row prunes it
-// to exactly k entries with a two-key radix select (8-bit digits on the
-// score key, then on the index for ties at the boundary) and raises the
-// threshold to the new k-th entry.  At the end the survivors are sorted
-// by index and written.
+// A row is owned by a group of NT threads (NW = NT/32 warps).  Its
+// candidate buffer of `cap` (key, index) pairs is split into NW
+// sub-buffers, one per warp, so a warp appends with a ballot and a count
+// it keeps in a register -- no atomics.  Callers feed each warp its keys in
+// ascending token order, so every sub-buffer stays sorted by index.  An
+// arriving pair is appended iff it ranks above the row's admission
+// threshold (the current k-th candidate).  When a sub-buffer nears its
+// share the group prunes the row to exactly k entries: a radix select over
+// the order-preserving score key that starts at the highest bit where the
+// candidates differ (8-bit digits, per-warp histograms), then over the
+// index for ties at the boundary.  Each warp compacts its own survivors in
+// place, in order (coalesced, and the sub-buffers stay sorted); only if one
+// warp would keep too many to leave room for further appends are the
+// survivors dealt round-robin across the sub-buffers (the row is then no
+// longer sorted).  The threshold rises to the new k-th entry.  At the end a
+// sorted row is written by merging its sub-buffers (each entry's output
+// position is its rank in its own list plus binary-searched ranks in the
+// others); an unsorted row is bitonic-sorted.
 //
-// The buffer may live in shared or global memory (generic pointers).
+// Buffers may live in shared or global memory (generic pointers).
 #pragma once
 
 #include "dsa_common.cuh"
 
 namespace dsa {
 
-static constexpr int kCandCap = 4096;  // candidates per row buffer
+static constexpr int kCandCap = 4096;  // largest candidate buffer per row
 
 struct TopkRowState {  // shared memory, one per row in flight
-    int count;
     uint32_t thr_key;  // admit (key, idx) iff key > thr_key || (key == thr_key && idx < thr_idx)
     int thr_idx;
+    int cnt[4];        // per-warp sub-buffer counts, published at check points
+    int sorted;        // 1 while every sub-buffer is in ascending index order
     int pad;
 };
 
-struct TopkScratch {  // shared memory, one per selection group
-    int hist[256];
-    int warp_val[16];
+template <int NW>
+struct TopkScratchT {  // shared memory, one per selection group
+    int hist[NW][256];
+    int warp_val[NW];
     int sel_digit, sel_above, sel_equal, misc;
 };
 
 __device__ __forceinline__ void topk_row_init(TopkRowState* st) {
-    st->count = 0;
     st->thr_key = 0u;
     st->thr_idx = 0x7fffffff;
+    st->cnt[0] = st->cnt[1] = st->cnt[2] = st->cnt[3] = 0;
+    st->sorted = 1;
 }
 
-__device__ __forceinline__ bool topk_admit(const TopkRowState* st, uint32_t key, int idx) {
-    const uint32_t tk = st->thr_key;
-    return key > tk || (key == tk && idx < st->thr_idx);
-}
-
-// Warp-aggregated append into a buffer of `cap` entries.  Every lane of
-// the warp must call it.  Callers prune before a buffer can fill; an append
-// past `cap` is dropped and flagged instead of written.
-__device__ __forceinline__ void topk_append_warp(TopkRowState* st, uint32_t* ckey, int* cidx, uint32_t key,
-                                                 int idx, bool admit, int cap, WsHeader* hdr) {
+// Warp append into this warp's sub-buffer (`sub` entries at ckey/cidx).
+// Every lane of the warp must call it; `cnt` is the warp's (uniform) count.
+// Entries past the sub-buffer are dropped (callers prune before that can
+// happen); `cnt` still counts them, so the caller can report an overflow.
+__device__ __forceinline__ void topk_append_warp(uint32_t* ckey, int* cidx, int& cnt, uint32_t key, int idx,
+                                                 bool admit, int sub) {
     const unsigned m = __ballot_sync(0xffffffffu, admit);
-    if (m == 0u) return;
-    const int lane = threadIdx.x & 31;
-    const int leader = __ffs(m) - 1;
-    int base = 0;
-    if (lane == leader) base = atomicAdd(&st->count, __popc(m));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (admit) {
-        const int pos = base + __popc(m & ((1u << lane) - 1u));
-        if (pos < cap) {
-            ckey[pos] = key;
-            cidx[pos] = idx;
-        } else {
-            raise_status(hdr, DSA_STATUS_OVERFLOW, pos);
-        }
-    }
+    const int pos = cnt + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
+    const uint32_t doit = static_cast<uint32_t>(admit & (pos < sub));
+    // predicated stores: no divergent branch around them
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %0, 0;\n\t"
+        "@p st.u32 [%1], %3;\n\t"
+        "@p st.u32 [%2], %4;\n\t}" ::"r"(doit),
+        "l"(ckey + pos), "l"(cidx + pos), "r"(key), "r"(idx)
+        : "memory");
+    cnt += __popc(m);
 }
 
 template <int NT>
 struct TopkGroup {
-    static_assert(NT % 32 == 0 && NT <= 512, "group of whole warps");
-    static constexpr int PER = kCandCap / NT;
+    static constexpr int NW = NT / 32;
+    static constexpr int PER = kCandCap / NT;  // items per thread when a row is loaded
+    static_assert(NT % 32 == 0 && NW <= 4, "group of at most 4 warps");
     static_assert(PER <= 32, "per-thread item mask is 32 bits");
+    using Scratch = TopkScratchT<NW>;
 
     int tid;   // thread index within the group
     int bar;   // named barrier id reserved for the group
-    TopkScratch* sc;
-    int cap;   // entries in each row buffer (<= kCandCap)
+    Scratch* sc;
+    int cap;   // entries in each row buffer (<= kCandCap, a multiple of NT)
 
     __device__ __forceinline__ void sync() const { named_bar_sync(bar, NT); }
+    __device__ __forceinline__ int sub() const { return cap / NW; }
+    __device__ __forceinline__ int warp() const { return tid >> 5; }
 
-    // kk-th largest (1-based) of the participating items v[i] (bit i of
-    // `part`) over the whole group.  Returns it; n_greater / n_equal count
-    // the participating items above / equal to it.
+    __device__ int sum_reduce(int x) const {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if ((tid & 31) == 0) sc->warp_val[tid >> 5] = x;
+        sync();
+        int r = 0;
+#pragma unroll
+        for (int j = 0; j < NW; ++j) r += sc->warp_val[j];
+        sync();
+        return r;
+    }
+    __device__ uint32_t umax_reduce(uint32_t x) const {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) x = max(x, __shfl_xor_sync(0xffffffffu, x, off));
+        if ((tid & 31) == 0) sc->warp_val[tid >> 5] = static_cast<int>(x);
+        sync();
+        uint32_t r = 0u;
+#pragma unroll
+        for (int j = 0; j < NW; ++j) r = max(r, static_cast<uint32_t>(sc->warp_val[j]));
+        sync();
+        return r;
+    }
+
+    // kk-th largest (1-based, kk <= number of participants) of the
+    // participating items v[i] (bit i of `part`) over the whole group.
+    // n_greater / n_equal count the participants above / equal to it.
     __device__ uint32_t kth_largest(const uint32_t (&v)[PER], uint32_t part, int kk, int& n_greater,
                                     int& n_equal) const {
-        uint32_t prefix = 0u, fixed = 0u;
+        // the digits start at the highest bit where participants differ
+        uint32_t hi = 0u, lo_inv = 0u;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            if ((part >> i) & 1u) {
+                hi = max(hi, v[i]);
+                lo_inv = max(lo_inv, ~v[i]);
+            }
+        }
+        hi = umax_reduce(hi);
+        const uint32_t lo = ~umax_reduce(lo_inv);
+        const uint32_t diff = hi ^ lo;
+        if (diff == 0u) {  // every participant is equal
+            n_greater = 0;
+            n_equal = sum_reduce(__popc(part));
+            return hi;
+        }
+        int nbits = 32 - __clz(diff);  // bits below the common prefix
+        uint32_t fixed = nbits >= 32 ? 0u : ~((1u << nbits) - 1u);
+        uint32_t prefix = hi & fixed;
         int above = 0, equal = 0;
+        const int w = warp();
 #pragma unroll 1
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            for (int b = tid; b < 256; b += NT) sc->hist[b] = 0;
+        while (nbits > 0) {
+            const int width = nbits < 8 ? nbits : 8;
+            const int shift = nbits - width;
+            const uint32_t dmask = (1u << width) - 1u;
+            for (int b = tid; b < NW * 256; b += NT) (&sc->hist[0][0])[b] = 0;
             sync();
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
-                if (((part >> i) & 1u) && (v[i] & fixed) == prefix)
-                    atomicAdd(&sc->hist[(v[i] >> shift) & 255u], 1);
+                if (((part >> i) & 1u) && (v[i] & fixed) == prefix) atomicAdd(&sc->hist[w][(v[i] >> shift) & dmask], 1);
             }
             sync();
             if (tid < 32) {
                 const int lane = tid;
+                int cnt8[8];
                 int s8 = 0;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) s8 += sc->hist[lane * 8 + j];
+                for (int j = 0; j < 8; ++j) {
+                    int c = 0;
+#pragma unroll
+                    for (int ww = 0; ww < NW; ++ww) c += sc->hist[ww][lane * 8 + j];
+                    cnt8[j] = c;
+                    s8 += c;
+                }
                 int suf = s8;  // count in bins >= lane*8
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -116,15 +176,16 @@ struct TopkGroup {
                 const int L = 31 - __clz(ball);
                 if (lane == L) {
                     int acc = suf - s8;
+                    bool found = false;
+#pragma unroll
                     for (int j = 7; j >= 0; --j) {
-                        const int c = sc->hist[L * 8 + j];
-                        if (acc + c >= kk) {
+                        if (!found && acc + cnt8[j] >= kk) {
                             sc->sel_digit = L * 8 + j;
                             sc->sel_above = acc;
-                            sc->sel_equal = c;
-                            break;
+                            sc->sel_equal = cnt8[j];
+                            found = true;
                         }
-                        acc += c;
+                        acc += cnt8[j];
                     }
                 }
             }
@@ -134,7 +195,8 @@ struct TopkGroup {
             above += sc->sel_above;
             equal = sc->sel_equal;
             prefix |= static_cast<uint32_t>(dsel) << shift;
-            fixed |= 0xFFu << shift;
+            fixed |= dmask << shift;
+            nbits = shift;
         }
         n_greater = above;
         n_equal = equal;
@@ -154,7 +216,7 @@ struct TopkGroup {
         sync();
         int before = 0, tot = 0;
 #pragma unroll
-        for (int j = 0; j < NT / 32; ++j) {
+        for (int j = 0; j < NW; ++j) {
             const int x = sc->warp_val[j];
             before += (j < w) ? x : 0;
             tot += x;
@@ -171,29 +233,45 @@ struct TopkGroup {
         sync();
         int r = sc->warp_val[0];
 #pragma unroll
-        for (int j = 1; j < NT / 32; ++j) r = max(r, sc->warp_val[j]);
+        for (int j = 1; j < NW; ++j) r = max(r, sc->warp_val[j]);
         sync();
         return r;
     }
 
-    // Keep exactly the k best candidates of the row (requires count > k).
-    // All NT threads call it; st->count is read after a group barrier.
-    __device__ void prune(TopkRowState* st, uint32_t* ckey, int* cidx, int k) const {
-        const int n = min(st->count, cap);
-        if (n <= k) return;  // nothing to drop (every thread reads the same n)
-        uint32_t rk[PER];
-        int ri[PER];
-        uint32_t valid = 0u;
+    // This thread's share of the row: entries lane, lane+32, ... of its warp's sub-buffer.
+    __device__ void load_own(const TopkRowState* st, const uint32_t* ckey, const int* cidx, uint32_t (&rk)[PER],
+                             int (&ri)[PER], uint32_t& valid) const {
+        const int w = warp(), lane = tid & 31, s = sub();
+        const int n = min(st->cnt[w], s);
+        const uint32_t* kk = ckey + w * s;
+        const int* ii = cidx + w * s;
+        valid = 0u;
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int j = tid + i * NT;
+            const int j = lane + 32 * i;
             const bool ok = j < n;
-            rk[i] = ok ? ckey[j] : 0u;
-            ri[i] = ok ? cidx[j] : 0;
+            rk[i] = ok ? kk[j] : 0u;
+            ri[i] = ok ? ii[j] : 0;
             valid |= (ok ? 1u : 0u) << i;
         }
+    }
+
+    // Keep exactly the k best candidates of the row and raise the threshold.
+    // A warp keeps its survivors in its own sub-buffer, in order, when every
+    // warp keeps at most `keep_max`; otherwise they are dealt round-robin.
+    // All NT threads call it after a group barrier that follows the
+    // publication of st->cnt.
+    __device__ void prune(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int keep_max) const {
+        int total0 = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) total0 += min(st->cnt[w], sub());
+        if (total0 <= k) return;  // nothing to drop (every thread reads the same counts)
+        uint32_t rk[PER];
+        int ri[PER];
+        uint32_t valid;
+        load_own(st, ckey, cidx, rk, ri, valid);
         int G, E;
-        const uint32_t kstar = kth_largest(rk, valid, k, G, E);  // includes barriers: loads are done
+        const uint32_t kstar = kth_largest(rk, valid, k, G, E);  // barriers inside: all loads are done
         const int kk = k - G;  // entries needed from key == kstar
         uint32_t eq = 0u;
 #pragma unroll
@@ -215,40 +293,135 @@ struct TopkGroup {
             keep |= ((gt || ke) ? 1u : 0u) << i;
             if (ke) maxeq = max(maxeq, ri[i]);
         }
-        int total;
-        int pos = excl_scan(__popc(keep), &total);  // barrier inside: every load above is done
+        const int w = warp(), lane = tid & 31, s = sub();
+        const unsigned lt = (1u << lane) - 1u;
+        // this warp's survivors, counted in sub-buffer order
+        int wkeep = 0;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            if ((keep >> i) & 1u) {
-                ckey[pos] = rk[i];
-                cidx[pos] = ri[i];
-                ++pos;
+        for (int i = 0; i < PER; ++i) wkeep += __popc(__ballot_sync(0xffffffffu, (keep >> i) & 1u));
+        if (lane == 0) sc->warp_val[w] = wkeep;
+        sync();  // every load above is done before any store below
+        int wmax = 0, total = 0;
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) {
+            wmax = max(wmax, sc->warp_val[ww]);
+            total += sc->warp_val[ww];
+        }
+        sync();
+        if (wmax <= keep_max) {
+            // compact in place, in order: coalesced and still sorted by index
+            int b = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const unsigned m = __ballot_sync(0xffffffffu, (keep >> i) & 1u);
+                if ((keep >> i) & 1u) {
+                    const int pos = b + __popc(m & lt);
+                    ckey[w * s + pos] = rk[i];
+                    cidx[w * s + pos] = ri[i];
+                }
+                b += __popc(m);
+            }
+        } else {
+            // one warp holds too many survivors to keep appending: deal them round-robin
+            int tot2;
+            int r = excl_scan(__popc(keep), &tot2);
+            // indices of a row are unique, so exactly k survive; clamp anyway so that
+            // corrupt input can never overfill a buffer
+            total = min(tot2, k);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                if (((keep >> i) & 1u) && r < total) {
+                    const int ww = r % NW, slot = r / NW;
+                    ckey[ww * s + slot] = rk[i];
+                    cidx[ww * s + slot] = ri[i];
+                    ++r;
+                }
             }
         }
         const int thr_idx = max_reduce(maxeq);
         if (tid == 0) {
-            st->count = total;  // == k
             st->thr_key = kstar;
             st->thr_idx = thr_idx;
+        }
+        if (wmax <= keep_max) {
+            if (lane == 0) st->cnt[w] = wkeep;
+        } else if (tid == 0) {
+#pragma unroll
+            for (int ww = 0; ww < NW; ++ww) st->cnt[ww] = (total - ww + NW - 1) / NW;
+            st->sorted = 0;
         }
         sync();
     }
 
-    // Final selection of the row: prune to k if needed, sort the indices
-    // ascending in `sortbuf` (shared, >= next_pow2(k) ints) and write
-    // out[0..k) (then -1 padding).  All NT threads call it.
+    // Number of entries of the ascending list a[0..n) that are < x.
+    __device__ static __forceinline__ int lower_rank(const int* a, int n, int x) {
+        int lo = 0, hi = n;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (a[mid] < x)
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        return lo;
+    }
+
+    // Final selection of the row: prune to k if needed, then write the
+    // survivors ascending to out[0..k) (then -1 padding), using `sortbuf`
+    // (shared, >= next_pow2(k) ints).  All NT threads call it after a group
+    // barrier that follows the publication of st->cnt.
     __device__ void finish(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int* out, int* sortbuf) const {
+        prune(st, ckey, cidx, k, sub());
+        const int w = warp(), lane = tid & 31, s = sub();
+        if (st->sorted) {
+            // concatenate the NW ascending lists in sortbuf, then place every entry at
+            // its rank in its own list plus its ranks in the other lists
+            int off[NW + 1];
+            off[0] = 0;
+#pragma unroll
+            for (int ww = 0; ww < NW; ++ww) off[ww + 1] = off[ww] + min(min(st->cnt[ww], s), k - off[ww]);
+            const int n = off[NW];
+            for (int j = lane; j < off[w + 1] - off[w]; j += 32) sortbuf[off[w] + j] = cidx[w * s + j];
+            sync();
+            for (int e = tid; e < n; e += NT) {
+                int le = 0;
+#pragma unroll
+                for (int ww = 1; ww < NW; ++ww) le += (e >= off[ww]) ? 1 : 0;
+                const int x = sortbuf[e];
+                int pos = e - off[le];
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww)
+                    if (ww != le) pos += lower_rank(sortbuf + off[ww], off[ww + 1] - off[ww], x);
+                if (pos < k) out[pos] = x;
+            }
+            for (int j = n + tid; j < k; j += NT) out[j] = -1;
+            sync();
+            return;
+        }
+        uint32_t rk[PER];
+        int ri[PER];
+        uint32_t valid;
+        load_own(st, ckey, cidx, rk, ri, valid);
+        int n;
+        int r = excl_scan(__popc(valid), &n);
+        n = min(n, k);  // never more than k (and the sort buffer holds next_pow2(k))
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+            if (((valid >> i) & 1u) && r < n) sortbuf[r++] = ri[i];
+        int P = 1, lp = 0;
+        while (P < n) {
+            P <<= 1;
+            ++lp;
+        }
+        for (int j = n + tid; j < P; j += NT) sortbuf[j] = 0x7fffffff;
         sync();
-        if (st->count > k) prune(st, ckey, cidx, k);
-        const int n = min(st->count, k);
-        int P = 1;
-        while (P < n) P <<= 1;
-        for (int j = tid; j < P; j += NT) sortbuf[j] = (j < n) ? cidx[j] : 0x7fffffff;
-        sync();
-        for (int size = 2; size <= P; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        // bitonic sort of P = 2^lp entries, pair index i -> (lo, lo + stride)
+        for (int ls = 1; ls <= lp; ++ls) {
+            const int size = 1 << ls;
+            for (int lst = ls - 1; lst >= 0; --lst) {
+                const int stride = 1 << lst;
                 for (int i = tid; i < (P >> 1); i += NT) {
-                    const int lo = (i / stride) * stride * 2 + (i % stride);
+                    const int lo = ((i >> lst) << (lst + 1)) | (i & (stride - 1));
                     const int hi = lo + stride;
                     const int a = sortbuf[lo], b = sortbuf[hi];
                     const bool asc = (lo & size) == 0;

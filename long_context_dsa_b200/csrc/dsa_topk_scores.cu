@@ -15,7 +15,7 @@ struct TopkScoresSmem {
     uint32_t ckey[kCandCap];
     int cidx[kCandCap];
     int sortbuf[DSA_TOPK_MAX];
-    TopkScratch scratch;
+    TopkGroup<kTsThreads>::Scratch scratch;
     TopkRowState st;
 };
 
@@ -25,7 +25,10 @@ __global__ void __launch_bounds__(kTsThreads) topk_scores_kernel(const float* __
     extern __shared__ __align__(16) unsigned char smem_raw[];
     TopkScoresSmem& sm = *reinterpret_cast<TopkScoresSmem*>(smem_raw);
     TopkGroup<kTsThreads> grp{static_cast<int>(threadIdx.x), 1, &sm.scratch, kCandCap};
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int sub = grp.sub();
+    uint32_t* wkey = sm.ckey + w * sub;  // this warp's sub-buffer
+    int* widx = sm.cidx + w * sub;
 
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
         const int n = min(q_pos0 + r + 1, n_kv);
@@ -38,6 +41,9 @@ __global__ void __launch_bounds__(kTsThreads) topk_scores_kernel(const float* __
         grp.sync();
         const float* srow = scores + static_cast<long long>(r) * ld;
         int nan_seen = 0;
+        int cnt = 0;  // this warp's sub-buffer count (warp-uniform)
+        float thr_f = -INFINITY;
+        int thr_i = 0x7fffffff;
         for (int base = 0; base < n; base += kTsPerIter) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -45,16 +51,29 @@ __global__ void __launch_bounds__(kTsThreads) topk_scores_kernel(const float* __
                 const bool inb = j < n;
                 const float s = inb ? __ldg(srow + j) : 0.f;
                 nan_seen |= (inb && s != s);
-                const uint32_t key = score_key(s);
-                const bool adm = inb && topk_admit(&sm.st, key, j);
-                topk_append_warp(&sm.st, sm.ckey, sm.cidx, key, j, adm, kCandCap, hdr);
+                const bool adm = inb && (s > thr_f || (s == thr_f && j < thr_i));
+                topk_append_warp(wkey, widx, cnt, score_key(s), j, adm, sub);
             }
+            if (lane == 0) sm.st.cnt[w] = cnt;
+            if (cnt > sub && lane == 0) raise_status(hdr, DSA_STATUS_OVERFLOW, cnt);
             grp.sync();
-            const int c = sm.st.count;  // read by every thread before anyone appends again
-            grp.sync();
-            if (c > kCandCap - kTsPerIter) grp.prune(&sm.st, sm.ckey, sm.cidx, k);
+            int mx = 0, tot = 0;
+#pragma unroll
+            for (int ww = 0; ww < 4; ++ww) {
+                mx = max(mx, sm.st.cnt[ww]);
+                tot += sm.st.cnt[ww];
+            }
+            grp.sync();  // every thread has read the counts before any is rewritten
+            if (mx > sub - kTsPerIter / 4 && tot > k) {
+                grp.prune(&sm.st, sm.ckey, sm.cidx, k, sub - kTsPerIter / 4 - 32);
+                cnt = sm.st.cnt[w];
+                thr_f = key_score(sm.st.thr_key);
+                thr_i = sm.st.thr_idx;
+            }
         }
         if (nan_seen) raise_status(hdr, DSA_STATUS_NAN_SCORE, r);
+        if (lane == 0) sm.st.cnt[w] = cnt;
+        grp.sync();
         grp.finish(&sm.st, sm.ckey, sm.cidx, k, orow, sm.sortbuf);
     }
 }
