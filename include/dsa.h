@@ -186,8 +186,8 @@ DSA_API int idx_cache_get(const dsa_index_cache* cache, int layer, const char* p
  *       first d_v dims).
  *   idx [B, n_q, topk] int32
  *   O   [B, n_q, Hq, d_v]   fp32 (o_dtype DSA_F32) or bf16 (DSA_BF16)
- * Supported: d_qk == d_v in {64, 128} with Hq/Hkv in {1,2,4,8,16};
- * latent d_qk = 576, d_v = 512, Hkv = 1.
+ * Supported: d_qk == d_v in {64, 128} with Hq/Hkv in {1,2,4,8};
+ * latent d_qk = 576, d_v = 512, Hkv = 1, Hq a multiple of 8.
  * ====================================================================== */
 DSA_API int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, int d_qk, int d_v,
                                     int topk, size_t* bytes);

@@ -94,7 +94,7 @@ int check_attn_shape(const void* V, int B, int n_q, int n_kv, int Hq, int Hkv, i
     if (V == nullptr) {
         if (!(d_qk == 576 && d_v == 512 && Hkv == 1))
             return fail(DSA_ERR_UNSUPPORTED, "latent form needs d_qk=576, d_v=512, Hkv=1");
-        if (Hq % 16 != 0) return fail(DSA_ERR_UNSUPPORTED, "latent form needs Hq a multiple of 16");
+        if (Hq % 8 != 0) return fail(DSA_ERR_UNSUPPORTED, "latent form needs Hq a multiple of 8");
         return DSA_OK;
     }
     if (d_qk != d_v) return fail(DSA_ERR_UNSUPPORTED, "d_qk != d_v needs the latent form");

@@ -1,12 +1,271 @@
-// dsa_sparse_attn_latent.cu -- sparse attention over a shared latent KV row
-// (MLA-style: one 576-dim row per token is the key, its first 512 dims the
-// value).  Placeholder until the latent kernel lands: reports "no kernel".
+// dsa_sparse_attn_latent.cu -- sparse attention over a shared latent row per
+// token (MLA-style): the row's 576 dims are the key of every query head and
+// its first 512 dims the value.
+//
+// [Explainer] §稀疏注意力的隐性开销: each token attends only to its top-k
+// history tokens.  The latent layout itself is this library's reading for
+// the 1M-token configuration (the pages do not describe the KV layout).
+//
+// Design: one CTA per (query row, block of 8*WARPS query heads).  All warps
+// share the gathered rows: the CTA streams the selected tokens' latent rows
+// (1152 bytes each) through a cp.async ring, 16 tokens per stage, and every
+// warp computes its 8 heads on each stage with warp-level bf16 MMAs:
+// S^T = K Q^T (keys on M, the warp's 8 heads on N, K = 576) and
+// O^T += V^T P (d on M: 32 tiles of 16 for d_v = 512, kept in registers).
+// The query block is staged in shared memory once per row.  P moves into the
+// B-operand layout with movmatrix and is split into bf16 hi + lo parts.
 #include "dsa_common.cuh"
 
 namespace dsa {
 
-cudaError_t launch_sparse_attn_latent(const void*, const void*, const int*, int, int, int, int, int, float, void*,
-                                      bool, WsHeader*, int, cudaStream_t) {
+namespace lat {
+
+constexpr int DQK = 576, DV = 512;
+constexpr int CHUNK = 16;                 // tokens per stage
+constexpr int STAGES = 4;
+constexpr int RS = DQK * 2 + 16;          // padded row stride (bank-conflict-free ldmatrix)
+constexpr int SEGS = DQK * 2 / 16;        // 72 16-byte segments per row
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int WARPS>
+struct Cfg {
+    static constexpr int HB = 8 * WARPS;  // query heads per CTA
+    static constexpr int Q_BYTES = HB * RS;
+    static constexpr int STAGE_BYTES = CHUNK * RS;
+    static constexpr size_t SMEM = Q_BYTES + static_cast<size_t>(STAGES) * STAGE_BYTES + STAGES * CHUNK * 4;
+};
+
+template <int WARPS, bool OUT_BF16>
+__global__ void __launch_bounds__(WARPS * 32, 1)
+    latent_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ KV,
+                       const int* __restrict__ idx, int B, int n_q, int n_kv, int Hq, int topk, float scale_log2,
+                       void* __restrict__ O, WsHeader* hdr) {
+    using C = Cfg<WARPS>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char* sq = smem;
+    unsigned char* ring = smem + C::Q_BYTES;
+    int* sidx = reinterpret_cast<int*>(ring + STAGES * C::STAGE_BYTES);
+    const uint32_t sq_s = smem_u32(sq), ring_s = smem_u32(ring);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nthr = WARPS * 32;
+    const int hblocks = Hq / C::HB;
+    const long long units = static_cast<long long>(B) * n_q * hblocks;
+    const int nchunks = (topk + CHUNK - 1) / CHUNK;
+
+    const int qn = lane >> 2, hc = 2 * (lane & 3);
+    const int lrow = lane & 7, lq = lane >> 3;
+    const int k_key_off = ((lq & 1) ? 8 : 0) + lrow, k_d_off = (lq >= 2) ? 8 : 0;   // K: non-trans A
+    const int v_key_off = ((lq >= 2) ? 8 : 0) + lrow, v_d_off = (lq & 1) ? 8 : 0;  // V: trans A
+    // Q^T B fragments via ldmatrix.x4 over two k-steps: rows = heads, 8-element column groups
+    const int q_row = lane & 7, q_col = (lane >> 3) * 8;
+
+    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+        const long long row = u / hblocks;
+        const int hb = static_cast<int>(u % hblocks);
+        const long long b = row / n_q;
+        const int* irow = idx + row * topk;
+        const __nv_bfloat16* kvb = KV + static_cast<size_t>(b) * n_kv * DQK;
+
+        __syncthreads();  // the previous unit is done with the query block and the ring
+        // query block -> shared (its own cp.async group, retired with the first stage)
+        {
+            const __nv_bfloat16* qb = Q + (static_cast<size_t>(row) * Hq + hb * C::HB) * DQK;
+            for (int sgi = threadIdx.x; sgi < C::HB * SEGS; sgi += nthr) {
+                const int h = sgi / SEGS, sg = sgi % SEGS;
+                cp_async16(sq_s + h * RS + sg * 16, qb + static_cast<size_t>(h) * DQK + sg * 8, 16u);
+            }
+        }
+        auto issue = [&](int c) {
+            if (c < nchunks) {
+                const int s = c % STAGES;
+                if (threadIdx.x < CHUNK) {
+                    const int kk = c * CHUNK + threadIdx.x;
+                    int t = kk < topk ? __ldg(irow + kk) : -1;
+                    if (t < -1 || t >= n_kv) {
+                        raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
+                        t = -1;
+                    }
+                    sidx[s * CHUNK + threadIdx.x] = t;
+                }
+                for (int sgi = threadIdx.x; sgi < CHUNK * SEGS; sgi += nthr) {
+                    const int key = sgi / SEGS, sg = sgi % SEGS;
+                    const int kk = c * CHUNK + key;
+                    int t = kk < topk ? __ldg(irow + kk) : -1;
+                    const bool ok = t >= 0 && t < n_kv;
+                    cp_async16(ring_s + s * C::STAGE_BYTES + key * RS + sg * 16,
+                               kvb + static_cast<size_t>(ok ? t : 0) * DQK + sg * 8, ok ? 16u : 0u);
+                }
+            }
+            cp_async_commit();
+        };
+
+        float o[DV / 16][4];
+#pragma unroll
+        for (int i = 0; i < DV / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
+        const uint32_t qw = sq_s + (warp * 8 + q_row) * RS + q_col * 2;  // this lane's ldmatrix row of Q
+
+#pragma unroll
+        for (int c = 0; c < STAGES - 1; ++c) issue(c);
+        for (int c = 0; c < nchunks; ++c) {
+            issue(c + STAGES - 1);
+            cp_async_wait<STAGES - 1>();
+            __syncthreads();
+            const int s = c % STAGES;
+            const uint32_t kst = ring_s + s * C::STAGE_BYTES;
+            const int* si = sidx + s * CHUNK;
+            // ---- S^T = K Q^T over 36 k-steps (two per ldmatrix.x4 of Q)
+            float sacc[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t abase = kst + k_key_off * RS + k_d_off * 2;
+#pragma unroll 6
+            for (int kp = 0; kp < DQK / 32; ++kp) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(qw + kp * 64, b0, b1, b2, b3);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(abase + kp * 64, a0, a1, a2, a3);
+                mma_bf16(sacc, a0, a1, a2, a3, b0, b1);
+                ldsm_x4(abase + kp * 64 + 32, a0, a1, a2, a3);
+                mma_bf16(s2, a0, a1, a2, a3, b2, b3);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[e] += s2[e];
+            // ---- mask, scale, online softmax
+            const bool v0 = si[qn] >= 0, v1 = si[qn + 8] >= 0;
+            float mx[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                sacc[j] = v0 ? sacc[j] * scale_log2 : -INFINITY;
+                sacc[2 + j] = v1 ? sacc[2 + j] * scale_log2 : -INFINITY;
+                mx[j] = fmaxf(sacc[j], sacc[2 + j]);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
+            }
+            float alpha[2], mnew[2], p[4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                mnew[j] = fmaxf(mrun[j], mx[j]);
+                alpha[j] = (mnew[j] == -INFINITY) ? 1.f : exp2f(mrun[j] - mnew[j]);
+                mrun[j] = mnew[j];
+                p[j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[j] - mnew[j]);
+                p[2 + j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[2 + j] - mnew[j]);
+                lrun[j] = lrun[j] * alpha[j] + p[j] + p[2 + j];
+            }
+            const uint32_t h01 = pack_bf16(p[0], p[1]), h23 = pack_bf16(p[2], p[3]);
+            const __nv_bfloat162 hh01 = *reinterpret_cast<const __nv_bfloat162*>(&h01);
+            const __nv_bfloat162 hh23 = *reinterpret_cast<const __nv_bfloat162*>(&h23);
+            const uint32_t phi0 = movm_t(h01), phi1 = movm_t(h23);
+            const uint32_t plo0 = movm_t(pack_bf16(p[0] - __low2float(hh01), p[1] - __high2float(hh01)));
+            const uint32_t plo1 = movm_t(pack_bf16(p[2] - __low2float(hh23), p[3] - __high2float(hh23)));
+            // ---- O^T = alpha * O^T + V^T P  (V = first 512 dims of the latent rows)
+            const uint32_t vbase = kst + v_key_off * RS + v_d_off * 2;
+#pragma unroll
+            for (int dt = 0; dt < DV / 16; ++dt) {
+                o[dt][0] *= alpha[0];
+                o[dt][1] *= alpha[1];
+                o[dt][2] *= alpha[0];
+                o[dt][3] *= alpha[1];
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(vbase + dt * 32, a0, a1, a2, a3);
+                mma_bf16(o[dt], a0, a1, a2, a3, phi0, phi1);
+                mma_bf16(o[dt], a0, a1, a2, a3, plo0, plo1);
+            }
+            __syncthreads();  // stage s may be refilled
+        }
+        cp_async_wait<0>();
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) lrun[j] += __shfl_xor_sync(0xffffffffu, lrun[j], off);
+        }
+        const float inv0 = lrun[0] > 0.f ? 1.f / lrun[0] : 0.f;
+        const float inv1 = lrun[1] > 0.f ? 1.f / lrun[1] : 0.f;
+#pragma unroll
+        for (int dt = 0; dt < DV / 16; ++dt) {
+            const int d0 = dt * 16 + qn;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = hb * C::HB + warp * 8 + hc + j;
+                const float inv = j ? inv1 : inv0;
+                const size_t ob = (static_cast<size_t>(row) * Hq + h) * DV;
+                if (OUT_BF16) {
+                    __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(O) + ob;
+                    op[d0] = __float2bfloat16_rn(o[dt][j] * inv);
+                    op[d0 + 8] = __float2bfloat16_rn(o[dt][2 + j] * inv);
+                } else {
+                    float* op = reinterpret_cast<float*>(O) + ob;
+                    op[d0] = o[dt][j] * inv;
+                    op[d0 + 8] = o[dt][2 + j] * inv;
+                }
+            }
+        }
+    }
+}
+
+template <int WARPS>
+cudaError_t launch_w(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv, int Hq, int topk,
+                     float scale, void* O, bool out_bf16, WsHeader* hdr, int num_sms, cudaStream_t stream) {
+    using Cf = Cfg<WARPS>;
+    auto kern = out_bf16 ? latent_attn_kernel<WARPS, true> : latent_attn_kernel<WARPS, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cf::SMEM));
+    if (e != cudaSuccess) return e;
+    const long long units = static_cast<long long>(B) * n_q * (Hq / Cf::HB);
+    long long grid = num_sms;
+    if (grid > units) grid = units;
+    if (grid < 1) grid = 1;
+    kern<<<static_cast<int>(grid), WARPS * 32, Cf::SMEM, stream>>>(
+        static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(KV), idx, B, n_q, n_kv, Hq, topk,
+        scale * 1.4426950408889634f, O, hdr);
+    return cudaGetLastError();
+}
+
+}  // namespace lat
+
+cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
+                                      int Hq, int topk, float scale, void* O, bool out_bf16, WsHeader* hdr,
+                                      int num_sms, cudaStream_t stream) {
+    if (Hq % 64 == 0)
+        return lat::launch_w<8>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+    if (Hq % 32 == 0)
+        return lat::launch_w<4>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+    if (Hq % 16 == 0)
+        return lat::launch_w<2>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+    if (Hq % 8 == 0)
+        return lat::launch_w<1>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }
 

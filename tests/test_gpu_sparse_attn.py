@@ -105,3 +105,28 @@ def test_bf16_output():
     # half a bf16 ulp of the reference on top of the fp32 bar
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
     assert np.all(np.abs(O - ref) <= 2e-3 + 0.5 * ulp)
+
+
+# latent (MLA-style) form: one 576-dim row per token is the key, its first 512 dims the value
+LATENT = [
+    ("latent_h64", 1, 300, 0, 300, 64, 128, None),
+    ("latent_h16_chunk_b2", 2, 100, 400, 500, 16, 300, None),
+    ("latent_h8_k64", 1, 200, 0, 200, 8, 64, None),
+    ("latent_h64_k2048", 1, 2600, 0, 2600, 64, 2048, 48),
+]
+
+
+@pytest.mark.parametrize("case", LATENT, ids=[c[0] for c in LATENT])
+def test_latent_attention_matches_oracle(case):
+    name, B, n_q, q_pos0, n_kv, Hq, k, sample = case
+    Q, KV, _ = synth.attention_inputs(name, 0, B, n_q, n_kv, Hq, 1, 576, None)
+    idx = _indices(n_kv, k, 8, q_pos0, n_q, B)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    O = dsa.sparse_attn_topk(Q.to(DEV), KV.to(DEV), None, torch.from_numpy(idx).to(DEV), d_v=512, workspace=ws)
+    assert dsa.read_status(ws) == 0
+    O = O.cpu().numpy()
+    rows = np.arange(n_q) if sample is None else np.unique(np.concatenate(
+        [np.arange(4), np.arange(n_q - 4, n_q), np.random.default_rng(9).choice(n_q, sample, replace=False)]))
+    for b in range(B):
+        ref = oracle.sparse_attention(Q[b, rows], KV[b], None, idx[b, rows], d_v=512)
+        check_attention(O[b, rows], ref)
