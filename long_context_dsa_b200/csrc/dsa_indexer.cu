@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(320, 1)
                         for (int q = 0; q < C::QG; ++q) {
                             if ((need >> q) & 1ull) {
                                 uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
-                                grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk, room - 32);
+                                grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk, room - 32, sortbuf);
                             }
                         }
 #pragma unroll
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (qi >= p.n_q) break;
                 uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
                 grp.finish(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk,
-                           p.idx_out + (static_cast<size_t>(b) * p.n_q + qi) * p.topk, sortbuf);
+                           p.idx_out + (static_cast<size_t>(b) * p.n_q + qi) * p.topk, nullptr, sortbuf);
             }
         }
     }
@@ -500,12 +500,15 @@ cudaError_t launch_t(const void* q, const float* q_scale, const void* k, const f
 
 }  // namespace
 
+bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype);
+size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms);
+cudaError_t launch_indexer_decode(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int H,
+                                  int topk, int* idx_out, void* ws, int num_sms, cudaStream_t stream);
+
 size_t indexer_workspace_bytes(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype,
                                int num_sms) {
-    (void)q_pos0;
-    (void)n_kv;
-    (void)d;
-    (void)dtype;
+    if (indexer_decode_supported(B, n_q, q_pos0, n_kv, H, d, topk, dtype))
+        return indexer_decode_workspace_bytes(B, q_pos0, topk, num_sms);
     const int n_tiles = tiles_per_b(n_q, H) * B;
     const int grid = grid_for(n_tiles, num_sms);
     const size_t qg = 256 / H;
@@ -516,6 +519,9 @@ cudaError_t launch_indexer(const void* q, const float* q_scale, const void* k, c
                            int dtype, int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int* idx_out,
                            float* scores_out, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
     (void)ws_bytes;
+    // one query per sequence: the split decode kernel (the selection path only)
+    if (!scores_out && indexer_decode_supported(B, n_q, q_pos0, n_kv, H, d, topk, dtype))
+        return launch_indexer_decode(q, k, w, B, q_pos0, n_kv, H, topk, idx_out, ws, num_sms, stream);
 #define DSA_IDX_CASE(HH, DD, F8)                                                                              \
     if (H == HH && d == DD && (dtype == DSA_E4M3) == F8)                                                     \
         return launch_t<HH, DD, F8>(q, q_scale, k, k_scale, w, B, n_q, q_pos0, n_kv, topk, idx_out, scores_out, ws, \

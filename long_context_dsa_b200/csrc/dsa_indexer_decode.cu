@@ -1,0 +1,373 @@
+// dsa_indexer_decode.cu -- the fused indexer + top-k for decode: one query
+// per sequence against a long key cache.
+//
+// Same operation as dsa_indexer.cu (the DSA lightning indexer, [QbitAI]
+// §IndexCache; [Term] "dot product + top-k").  With one query row there is
+// no query reuse to harvest, so the work is a scan of the key cache at HBM
+// speed: the prefill kernel would give each sequence one CTA and pad each
+// MMA to 16 queries.  Here:
+//   * Each sequence's key range is split over several CTAs (units of
+//     (sequence, split)), so B*splits units cover all SMs.
+//   * The MMA is 128 keys x H_I heads (N = H_I, one query) and the 512 TMEM
+//     columns hold a ring of 512/H_I accumulators, so many key tiles are in
+//     flight while the epilogue drains older ones.
+//   * A 4-stage TMA ring streams the keys; the candidate buffer of the unit's
+//     single row lives in shared memory.
+//   * Each unit writes its partial top-k (ascending indices with their score
+//     keys); topk_merge_pairs then selects the final top-k of each sequence
+//     from its units' lists (dsa_topk_scores.cu).
+#include <cuda.h>
+
+#include "dsa_tc.cuh"
+#include "dsa_topk.cuh"
+
+namespace dsa {
+
+cudaError_t launch_topk_merge_pairs(const uint32_t* keys, const int* idxs, int rows, int len, int k, int* out,
+                                    WsHeader* hdr, int num_sms, cudaStream_t stream);
+
+template <int H>
+struct DecCfg {
+    static constexpr int N = H;              // accumulator columns: one query's heads
+    static constexpr int NACC = 512 / N;     // accumulators in flight
+    static constexpr int STAGES = 4;
+    static constexpr int A_STAGE = 128 * 256;  // 128 keys x 128 bf16
+    static constexpr int B_BYTES = N * 256;    // the query's H rows x 128 bf16
+    static constexpr int CAP = kCandCap;       // candidate buffer of the unit's row (shared memory)
+    static constexpr int THREADS = 192;        // warps 0-3 epilogue, 4 producer, 5 MMA
+    static constexpr int OFF_B = 0;
+    static constexpr int OFF_A = OFF_B + ((B_BYTES + 1023) / 1024) * 1024;
+    static constexpr int OFF_CK = OFF_A + STAGES * A_STAGE;
+    static constexpr int OFF_CI = OFF_CK + CAP * 4;
+    static constexpr int OFF_SORT = OFF_CI + CAP * 4;
+    static constexpr int OFF_W = OFF_SORT + DSA_TOPK_MAX * 4;
+    static constexpr int OFF_SC = OFF_W + 64 * 4;
+    static constexpr int OFF_ST = OFF_SC + static_cast<int>(sizeof(TopkGroup<128>::Scratch));
+    static constexpr int OFF_BAR = (OFF_ST + static_cast<int>(sizeof(TopkRowState)) + 7) / 8 * 8;
+    static constexpr int NBAR = 2 + 2 * STAGES + 2 * NACC;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct DecParams {
+    const float* w;
+    int B, q_pos0, n_kv, topk, splits, tiles_per_split;
+    uint32_t* part_key;  // [B * splits, topk]
+    int* part_idx;       // [B * splits, topk]
+    WsHeader* hdr;
+};
+
+template <int H>
+__global__ void __launch_bounds__(192, 1)
+    indexer_decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                          const DecParams p) {
+    using C = DecCfg<H>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    unsigned char* sB = smem + C::OFF_B;
+    unsigned char* sA = smem + C::OFF_A;
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + C::OFF_CK);
+    int* cidx = reinterpret_cast<int*>(smem + C::OFF_CI);
+    int* sortbuf = reinterpret_cast<int*>(smem + C::OFF_SORT);
+    float* ws = reinterpret_cast<float*>(smem + C::OFF_W);
+    auto* sc = reinterpret_cast<TopkGroup<128>::Scratch*>(smem + C::OFF_SC);
+    TopkRowState* st = reinterpret_cast<TopkRowState*>(smem + C::OFF_ST);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars + 0;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* kv_full = bars + 2;
+    uint64_t* kv_empty = kv_full + C::STAGES;
+    uint64_t* acc_full = kv_empty + C::STAGES;
+    uint64_t* acc_empty = acc_full + C::NACC;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+    int* wg_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);  // written only by the epilogue
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int units = p.B * p.splits;
+    const int nkt = (p.q_pos0 + 1 + 127) / 128;  // key tiles of a sequence (keys 0..q_pos0)
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int a = 0; a < C::NACC; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 128);
+        }
+        *abort_flag = 0;
+        *wg_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        tc::prefetch_tmap(&tmap_q);
+        tc::prefetch_tmap(&tmap_k);
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto unit_range = [&](int u, int& b, int& j0, int& j1) {
+        b = u / p.splits;
+        const int sp = u % p.splits;
+        j0 = sp * p.tiles_per_split;
+        j1 = min(nkt, j0 + p.tiles_per_split);
+    };
+
+    if (warp == 4) {
+        // ================================================== TMA producer
+        if (lane == 0) {
+            uint32_t it = 0, wt = 0;
+            bool ok = true;
+            int pend_q = -1;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++wt) {
+                int b, j0, j1;
+                unit_range(u, b, j0, j1);
+                if (wt > 0 && !mbar_wait(q_empty, (wt - 1) & 1)) { ok = false; break; }
+                mbar_arrive_expect_tx(q_full, C::B_BYTES);
+                for (int kb = 0; kb < 2; ++kb) tc::tma_load_2d(sB + kb * H * 128, &tmap_q, kb * 64, b * H, q_full);
+                pend_q = static_cast<int>(wt);
+                for (int j = j0; j < j1; ++j, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t rr = it / C::STAGES;
+                    if (rr > 0 && !mbar_wait(&kv_empty[s], (rr - 1) & 1)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&kv_full[s], C::A_STAGE);
+                    for (int kb = 0; kb < 2; ++kb)
+                        tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128, &tmap_k, kb * 64, b * p.n_kv + j * 128,
+                                        &kv_full[s]);
+                    if (*reinterpret_cast<volatile int*>(abort_flag)) { ok = false; ++it; break; }
+                }
+            }
+            if (!ok) {
+                raise_status(p.hdr, DSA_STATUS_TIMEOUT, 0x2d01);
+                atomicExch(abort_flag, 1);
+            }
+            if (pend_q >= 0) mbar_wait(q_full, pend_q & 1);
+            for (uint32_t k2 = (it > C::STAGES ? it - C::STAGES : 0); k2 < it; ++k2)
+                mbar_wait(&kv_full[k2 % C::STAGES], (k2 / C::STAGES) & 1);
+        }
+    } else if (warp == 5) {
+        // ================================================== MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::make_idesc(1, 1, 128, C::N);
+            uint32_t it = 0, wt = 0, ua = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++wt) {
+                int b, j0, j1;
+                unit_range(u, b, j0, j1);
+                (void)b;
+                if (!mbar_wait(q_full, wt & 1)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t b0 = smem_u32(sB);
+                for (int j = j0; j < j1; ++j, ++it, ++ua) {
+                    const int s = it % C::STAGES;
+                    const int a = ua % C::NACC;
+                    if (!mbar_wait(&kv_full[s], (it / C::STAGES) & 1)) { ok = false; break; }
+                    if (ua >= C::NACC && !mbar_wait(&acc_empty[a], ((ua / C::NACC) - 1) & 1)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t a0 = smem_u32(sA + s * C::A_STAGE);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t ad = tc::make_sdesc_sw128(a0 + (ks >> 2) * (128 * 128) + (ks & 3) * 32);
+                        const uint64_t bd = tc::make_sdesc_sw128(b0 + (ks >> 2) * (H * 128) + (ks & 3) * 32);
+                        tc::mma_f16(tmem_base + a * C::N, ad, bd, idesc, ks > 0);
+                    }
+                    tc::mma_commit(&acc_full[a]);
+                    tc::mma_commit(&kv_empty[s]);
+                    if (*reinterpret_cast<volatile int*>(abort_flag)) { ok = false; break; }
+                }
+                tc::mma_commit(q_empty);
+            }
+            if (!ok) {
+                raise_status(p.hdr, DSA_STATUS_TIMEOUT, 0x2d02);
+                atomicExch(abort_flag, 1);
+            }
+        }
+    } else {
+        // ================================================== epilogue (warps 0-3)
+        const int tid = threadIdx.x;  // key lane
+        TopkGroup<128> grp{tid, 1, sc, C::CAP};
+        const int sub = grp.sub();
+        constexpr int CHECK = 4;
+        const int room = sub - CHECK * 32;
+        const uint32_t tlane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        uint32_t ua = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int b, j0, j1;
+            unit_range(u, b, j0, j1);
+            if (tid < H) ws[tid] = p.w[static_cast<size_t>(b) * H + tid];
+            if (tid == 0) topk_row_init(st);
+            grp.sync();
+            int cnt = 0;
+            uint32_t* wkey = ckey + warp * sub;
+            int* widx = cidx + warp * sub;
+            for (int j = j0; j < j1; ++j, ++ua) {
+                const int a = ua % C::NACC;
+                const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[a], (ua / C::NACC) & 1));
+                float sc_v = 0.f;
+                if (got) {
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < H / 32; ++c) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(tlane + a * C::N + c * 32, v);
+                        tc::tmem_wait_ld_dep(v);
+                        unsigned long long a2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const unsigned long long w2 = *reinterpret_cast<const unsigned long long*>(ws + c * 32 + 2 * i);
+                            tc::fma2(a2[i & 3], w2,
+                                     tc::pack2(fmaxf(__uint_as_float(v[2 * i]), 0.f),
+                                               fmaxf(__uint_as_float(v[2 * i + 1]), 0.f)));
+                        }
+                        const float2 t = tc::unpack2(tc::add2(tc::add2(a2[0], a2[1]), tc::add2(a2[2], a2[3])));
+                        sc_v += t.x + t.y;
+                    }
+                    tc::fence_before_sync();
+                    mbar_arrive(&acc_empty[a]);
+                } else if (lane == 0) {
+                    raise_status(p.hdr, DSA_STATUS_TIMEOUT, 0x2d03);
+                    atomicExch(abort_flag, 1);
+                    *wg_abort = 1;
+                }
+                const int s_key = j * 128 + tid;
+                const uint32_t key = score_key(sc_v);
+                const uint32_t tk = st->thr_key;
+                const bool adm = got & (s_key <= p.q_pos0) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
+                topk_append_warp(wkey, widx, cnt, key, s_key, adm, sub);
+                if (((j - j0) % CHECK) == CHECK - 1 || j == j1 - 1) {
+                    if (lane == 0) st->cnt[warp] = cnt;
+                    grp.sync();
+                    int mx = 0, tot = 0;
+#pragma unroll
+                    for (int ww = 0; ww < 4; ++ww) {
+                        mx = max(mx, st->cnt[ww]);
+                        tot += st->cnt[ww];
+                    }
+                    const bool stop = *wg_abort != 0;  // read between two barriers: uniform
+                    grp.sync();
+                    if (stop) { ok = false; break; }
+                    if (mx > room && tot > p.topk) {
+                        grp.prune(st, ckey, cidx, p.topk, room - 32, sortbuf);
+                        cnt = st->cnt[warp];
+                    }
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) st->cnt[warp] = cnt;
+            grp.sync();
+            grp.finish(st, ckey, cidx, p.topk, p.part_idx + static_cast<size_t>(u) * p.topk,
+                       p.part_key + static_cast<size_t>(u) * p.topk, sortbuf);
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// ----------------------------------------------------------------- host side
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int dec_splits(int B, int nkt, int num_sms) {
+    int s = (2 * num_sms + B - 1) / B;
+    if (s > nkt / 8) s = nkt / 8;  // keep at least 8 key tiles per unit
+    if (s < 1) s = 1;
+    return s;
+}
+
+template <int H>
+cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int topk,
+                         int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
+    using C = DecCfg<H>;
+    CUtensorMap mq, mk;
+    if (!make_map_dec(&mq, q, static_cast<uint64_t>(B) * H, H) ||
+        !make_map_dec(&mk, k, static_cast<uint64_t>(B) * n_kv, 128))
+        return cudaErrorInvalidValue;
+    const int nkt = (q_pos0 + 1 + 127) / 128;
+    DecParams p;
+    p.w = w;
+    p.B = B;
+    p.q_pos0 = q_pos0;
+    p.n_kv = n_kv;
+    p.topk = topk;
+    p.splits = dec_splits(B, nkt, num_sms);
+    p.tiles_per_split = (nkt + p.splits - 1) / p.splits;
+    p.splits = (nkt + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty units
+    p.hdr = static_cast<WsHeader*>(ws);
+    const size_t parts = static_cast<size_t>(B) * p.splits * topk;
+    p.part_key = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kWsHeaderBytes);
+    p.part_idx = reinterpret_cast<int*>(p.part_key + parts);
+    auto kern = indexer_decode_kernel<H>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int units = B * p.splits;
+    kern<<<units < num_sms ? units : num_sms, C::THREADS, C::SMEM, stream>>>(mq, mk, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_topk_merge_pairs(p.part_key, p.part_idx, B, p.splits * topk, topk, idx_out, p.hdr, num_sms,
+                                   stream);
+}
+
+}  // namespace
+
+bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype) {
+    (void)B;
+    (void)n_kv;
+    (void)topk;
+    return n_q == 1 && d == 128 && dtype == DSA_BF16 && (H == 32 || H == 64) && q_pos0 + 1 >= 8 * 128;
+}
+
+size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms) {
+    const int nkt = (q_pos0 + 1 + 127) / 128;
+    int splits = dec_splits(B, nkt, num_sms);
+    const int tps = (nkt + splits - 1) / splits;
+    splits = (nkt + tps - 1) / tps;
+    return static_cast<size_t>(B) * splits * topk * 8;
+}
+
+cudaError_t launch_indexer_decode(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int H,
+                                  int topk, int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
+    if (H == 32) return launch_dec_t<32>(q, k, w, B, q_pos0, n_kv, topk, idx_out, ws, num_sms, stream);
+    if (H == 64) return launch_dec_t<64>(q, k, w, B, q_pos0, n_kv, topk, idx_out, ws, num_sms, stream);
+    return cudaErrorNotSupported;
+}
+
+}  // namespace dsa

@@ -18,11 +18,11 @@
 // index for ties at the boundary.  Each warp compacts its own survivors in
 // place, in order (coalesced, and the sub-buffers stay sorted); only if one
 // warp would keep too many to leave room for further appends are the
-// survivors dealt round-robin across the sub-buffers (the row is then no
-// longer sorted).  The threshold rises to the new k-th entry.  At the end a
-// sorted row is written by merging its sub-buffers (each entry's output
-// position is its rank in its own list plus binary-searched ranks in the
-// others); an unsorted row is bitonic-sorted.
+// survivors merged into index order and split evenly over the sub-buffers
+// (still sorted: later appends carry larger indices).  The threshold rises
+// to the new k-th entry.  At the end the row is written by merging its
+// sub-buffers: each entry's output position is its rank in its own list
+// plus its binary-searched ranks in the others.
 //
 // Buffers may live in shared or global memory (generic pointers).
 #pragma once
@@ -37,8 +37,6 @@ struct TopkRowState {  // shared memory, one per row in flight
     uint32_t thr_key;  // admit (key, idx) iff key > thr_key || (key == thr_key && idx < thr_idx)
     int thr_idx;
     int cnt[4];        // per-warp sub-buffer counts, published at check points
-    int sorted;        // 1 while every sub-buffer is in ascending index order
-    int pad;
 };
 
 template <int NW>
@@ -52,7 +50,6 @@ __device__ __forceinline__ void topk_row_init(TopkRowState* st) {
     st->thr_key = 0u;
     st->thr_idx = 0x7fffffff;
     st->cnt[0] = st->cnt[1] = st->cnt[2] = st->cnt[3] = 0;
-    st->sorted = 1;
 }
 
 // Warp append into this warp's sub-buffer (`sub` entries at ckey/cidx).
@@ -261,7 +258,7 @@ struct TopkGroup {
     // warp keeps at most `keep_max`; otherwise they are dealt round-robin.
     // All NT threads call it after a group barrier that follows the
     // publication of st->cnt.
-    __device__ void prune(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int keep_max) const {
+    __device__ void prune(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int keep_max, int* sortbuf) const {
         int total0 = 0;
 #pragma unroll
         for (int w = 0; w < NW; ++w) total0 += min(st->cnt[w], sub());
@@ -322,20 +319,37 @@ struct TopkGroup {
                 b += __popc(m);
             }
         } else {
-            // one warp holds too many survivors to keep appending: deal them round-robin
-            int tot2;
-            int r = excl_scan(__popc(keep), &tot2);
-            // indices of a row are unique, so exactly k survive; clamp anyway so that
-            // corrupt input can never overfill a buffer
-            total = min(tot2, k);
+            // one warp holds too many survivors to keep appending: merge all survivors into
+            // index order and split them evenly over the sub-buffers
+            int off[NW + 1];
+            off[0] = 0;
+            for (int ww = 0; ww < NW; ++ww) off[ww + 1] = off[ww] + sc_counts(ww);
+            int b = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {  // this warp's survivor indices, in order, into sortbuf
+                const unsigned m = __ballot_sync(0xffffffffu, (keep >> i) & 1u);
+                if (((keep >> i) & 1u) && off[w] + b + __popc(m & lt) < k) sortbuf[off[w] + b + __popc(m & lt)] = ri[i];
+                b += __popc(m);
+            }
+            sync();
+            total = min(total, k);
+            const int qn = (total + NW - 1) / NW;  // survivors per sub-buffer after the split
+            b = 0;
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
-                if (((keep >> i) & 1u) && r < total) {
-                    const int ww = r % NW, slot = r / NW;
-                    ckey[ww * s + slot] = rk[i];
-                    cidx[ww * s + slot] = ri[i];
-                    ++r;
+                const unsigned m = __ballot_sync(0xffffffffu, (keep >> i) & 1u);
+                if ((keep >> i) & 1u) {
+                    int r = b + __popc(m & lt);
+#pragma unroll
+                    for (int ww = 0; ww < NW; ++ww)
+                        if (ww != w) r += lower_rank(sortbuf + off[ww], min(off[ww + 1], k) - min(off[ww], k), ri[i]);
+                    if (r < total) {
+                        const int dw = r / qn, slot = r - dw * qn;
+                        ckey[dw * s + slot] = rk[i];
+                        cidx[dw * s + slot] = ri[i];
+                    }
                 }
+                b += __popc(m);
             }
         }
         const int thr_idx = max_reduce(maxeq);
@@ -346,12 +360,15 @@ struct TopkGroup {
         if (wmax <= keep_max) {
             if (lane == 0) st->cnt[w] = wkeep;
         } else if (tid == 0) {
+            const int qn = (total + NW - 1) / NW;
 #pragma unroll
-            for (int ww = 0; ww < NW; ++ww) st->cnt[ww] = (total - ww + NW - 1) / NW;
-            st->sorted = 0;
+            for (int ww = 0; ww < NW; ++ww) st->cnt[ww] = max(0, min(qn, total - ww * qn));
         }
         sync();
     }
+
+    // Survivor count of warp ww, as published in the scratch during prune.
+    __device__ __forceinline__ int sc_counts(int ww) const { return sc->warp_val[ww]; }
 
     // Number of entries of the ascending list a[0..n) that are < x.
     __device__ static __forceinline__ int lower_rank(const int* a, int n, int x) {
@@ -367,73 +384,41 @@ struct TopkGroup {
     }
 
     // Final selection of the row: prune to k if needed, then write the
-    // survivors ascending to out[0..k) (then -1 padding), using `sortbuf`
-    // (shared, >= next_pow2(k) ints).  All NT threads call it after a group
+    // survivors ascending by index to out_idx[0..k) (then -1 padding) and,
+    // if out_key is not NULL, their score keys to out_key (then 0).  Uses
+    // `sortbuf` (shared, >= k ints).  All NT threads call it after a group
     // barrier that follows the publication of st->cnt.
-    __device__ void finish(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int* out, int* sortbuf) const {
-        prune(st, ckey, cidx, k, sub());
+    __device__ void finish(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int* out_idx, uint32_t* out_key,
+                           int* sortbuf) const {
+        prune(st, ckey, cidx, k, sub(), sortbuf);
         const int w = warp(), lane = tid & 31, s = sub();
-        if (st->sorted) {
-            // concatenate the NW ascending lists in sortbuf, then place every entry at
-            // its rank in its own list plus its ranks in the other lists
-            int off[NW + 1];
-            off[0] = 0;
+        // concatenate the NW ascending lists in sortbuf, then place every entry at its rank
+        // in its own list plus its ranks in the other lists
+        int off[NW + 1];
+        off[0] = 0;
 #pragma unroll
-            for (int ww = 0; ww < NW; ++ww) off[ww + 1] = off[ww] + min(min(st->cnt[ww], s), k - off[ww]);
-            const int n = off[NW];
-            for (int j = lane; j < off[w + 1] - off[w]; j += 32) sortbuf[off[w] + j] = cidx[w * s + j];
-            sync();
-            for (int e = tid; e < n; e += NT) {
-                int le = 0;
-#pragma unroll
-                for (int ww = 1; ww < NW; ++ww) le += (e >= off[ww]) ? 1 : 0;
-                const int x = sortbuf[e];
-                int pos = e - off[le];
-#pragma unroll
-                for (int ww = 0; ww < NW; ++ww)
-                    if (ww != le) pos += lower_rank(sortbuf + off[ww], off[ww + 1] - off[ww], x);
-                if (pos < k) out[pos] = x;
-            }
-            for (int j = n + tid; j < k; j += NT) out[j] = -1;
-            sync();
-            return;
-        }
-        uint32_t rk[PER];
-        int ri[PER];
-        uint32_t valid;
-        load_own(st, ckey, cidx, rk, ri, valid);
-        int n;
-        int r = excl_scan(__popc(valid), &n);
-        n = min(n, k);  // never more than k (and the sort buffer holds next_pow2(k))
-#pragma unroll
-        for (int i = 0; i < PER; ++i)
-            if (((valid >> i) & 1u) && r < n) sortbuf[r++] = ri[i];
-        int P = 1, lp = 0;
-        while (P < n) {
-            P <<= 1;
-            ++lp;
-        }
-        for (int j = n + tid; j < P; j += NT) sortbuf[j] = 0x7fffffff;
+        for (int ww = 0; ww < NW; ++ww) off[ww + 1] = off[ww] + min(min(st->cnt[ww], s), k - off[ww]);
+        const int n = off[NW];
+        for (int j = lane; j < off[w + 1] - off[w]; j += 32) sortbuf[off[w] + j] = cidx[w * s + j];
         sync();
-        // bitonic sort of P = 2^lp entries, pair index i -> (lo, lo + stride)
-        for (int ls = 1; ls <= lp; ++ls) {
-            const int size = 1 << ls;
-            for (int lst = ls - 1; lst >= 0; --lst) {
-                const int stride = 1 << lst;
-                for (int i = tid; i < (P >> 1); i += NT) {
-                    const int lo = ((i >> lst) << (lst + 1)) | (i & (stride - 1));
-                    const int hi = lo + stride;
-                    const int a = sortbuf[lo], b = sortbuf[hi];
-                    const bool asc = (lo & size) == 0;
-                    if ((a > b) == asc) {
-                        sortbuf[lo] = b;
-                        sortbuf[hi] = a;
-                    }
-                }
-                sync();
+        for (int e = tid; e < n; e += NT) {
+            int le = 0;
+#pragma unroll
+            for (int ww = 1; ww < NW; ++ww) le += (e >= off[ww]) ? 1 : 0;
+            const int x = sortbuf[e];
+            int pos = e - off[le];
+#pragma unroll
+            for (int ww = 0; ww < NW; ++ww)
+                if (ww != le) pos += lower_rank(sortbuf + off[ww], off[ww + 1] - off[ww], x);
+            if (pos < k) {
+                out_idx[pos] = x;
+                if (out_key) out_key[pos] = ckey[le * s + (e - off[le])];
             }
         }
-        for (int j = tid; j < k; j += NT) out[j] = (j < n) ? sortbuf[j] : -1;
+        for (int j = n + tid; j < k; j += NT) {
+            out_idx[j] = -1;
+            if (out_key) out_key[j] = 0u;
+        }
         sync();
     }
 };

@@ -32,6 +32,9 @@ CASES = [
     ("h32_k16", 1, 1500, 0, 1500, 32, 128, 16, dict(r=32, base_std=1.0, noise_std=0.2)),
     ("h64_k1", 1, 600, 0, 600, 64, 128, 1, dict(r=32, base_std=1.0, noise_std=0.2)),
     ("h4_k3_b2", 2, 700, 0, 700, 4, 64, 3, dict(r=8, base_std=1 / 8, noise_std=1 / 8)),
+    # decode through the split kernel: long caches, one query per sequence, query inside the cache
+    ("decode_b2_h64", 2, 1, 19999, 20000, 64, 128, 2048, dict(r=32, base_std=1.0, noise_std=0.2)),
+    ("decode_mid_b4", 4, 1, 4000, 5000, 32, 128, 300, dict(r=32, base_std=1.0, noise_std=0.2)),
 ]
 
 
@@ -104,3 +107,18 @@ def test_indexer_repeatable():
     a = dsa.idx_score_topk(qd, kd, wd, k)
     b = dsa.idx_score_topk(qd, kd, wd, k)
     assert torch.equal(a, b)
+
+
+def test_indexer_survivors_concentrated_in_one_lane_range():
+    """Keys whose position mod 128 is below 32 (one epilogue warp's lanes) score far above the
+    rest, so one warp's candidate share holds most survivors and the prune must rebalance."""
+    B, L, H, d, k = 1, 6000, 32, 128, 2048
+    q, kk, w = _inputs("skew", B, L, 0, L, H, d, dict(r=32, base_std=1.0, noise_std=0.2))
+    hot = (torch.arange(L) % 128) < 32
+    kk = kk.float()
+    kk[:, hot] *= 4.0  # a longer key scores higher through the ReLU in expectation
+    kk = kk.to(torch.bfloat16)
+    idx = dsa.idx_score_topk(q.to(DEV), kk.to(DEV), w.to(DEV), k).cpu().numpy()[0]
+    ora = oracle.indexer_scores(q[0], kk[0], w[0])
+    frac = check_selection(idx, oracle.topk_select(ora, k), ora, 0, k, rtol=1e-3)
+    assert frac > 0.9

@@ -84,3 +84,17 @@ def test_nan_is_flagged():
     sc[2, 3] = np.nan
     _, bits = _run(sc, 2, 12)
     assert bits & dsa.STATUS_NAN_SCORE
+
+
+def test_survivors_concentrated_in_one_warp():
+    """High scores only where (position mod 128) < 32: one warp's share of the candidate buffer
+    fills with survivors, forcing the ordered rebalance inside the prune."""
+    n_kv, rows = 30000, 4
+    rng = np.random.default_rng(21)
+    sc = rng.standard_normal((rows, n_kv)).astype(np.float32)
+    hot = (np.arange(n_kv) % 128) < 32
+    sc[:, hot] += 10.0
+    for k in (2048, 1500):
+        got, bits = _run(sc, k, n_kv - rows)
+        assert bits == 0
+        assert np.array_equal(got, oracle.topk_select(sc, k, n_kv - rows))
