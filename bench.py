@@ -421,6 +421,123 @@ def run_profile_case(args):
                       "indexer_queries": nq_i, "attn_queries": nq_a, "n_kv": L}))
 
 
+def run_decode(args, dev):
+    """Decode step: 64 sequences, one new token each, at a 200000-token cache; 4 layers FSSS
+    (H_I=32, d_I=128, top-2048; attention 32 query / 4 KV heads, d=128)."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    B, Lc, pat = 64, 200000, "FSSS"
+    gen = synth.StructuredIndexer("decode200k", B, Lc, H_I, D_I, r=32, base_std=1.0, noise_std=0.2, device=dev,
+                                  seed=2000)
+    layers = []
+    for l in range(4):
+        Lh = {}
+        Lh["q_I"], Lh["w"] = gen.queries(l, Lc - 1, Lc)
+        Lh["k_I"] = gen.keys(l)
+        Lh["Q"], Lh["K"], Lh["V"] = synth.attention_inputs("decode200k", l, B, 1, Lc, HQ, HKV, DH, DH, device=dev,
+                                                           seed=2000)
+        Lh["O"] = torch.empty((B, 1, HQ, DH), dtype=torch.bfloat16, device=dev)
+        layers.append(Lh)
+    del gen
+    shape = dsa.group_shape(B, 1, Lc - 1, Lc, H_I, D_I, HQ, HKV, DH, DH, TOPK, o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((B, 1, TOPK), dtype=torch.int32, device=dev))
+    res = {}
+    for p in (pat, "FFFF"):
+        for _ in range(3):
+            dsa.layer_group_forward(shape, layers, p, cache, workspace=ws)
+        torch.cuda.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(12)]
+        for e in evs:
+            e.record()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 10
+        t0.record()
+        for _ in range(n - 1):
+            dsa.layer_group_forward(shape, layers, p, cache, workspace=ws)
+        dsa.layer_group_forward(shape, layers, p, cache, workspace=ws, events=evs)
+        t1.record()
+        torch.cuda.synchronize()
+        dsa.check_status(ws)
+        ms = t0.elapsed_time(t1) / n
+        idx_ms = sum(evs[3 * l].elapsed_time(evs[3 * l + 1]) for l in range(4))
+        att_ms = sum(evs[3 * l + 1].elapsed_time(evs[3 * l + 2]) for l in range(4))
+        res[p] = (ms, idx_ms, att_ms)
+    ms, idx_ms, att_ms = res[pat]
+    kbytes = B * Lc * D_I * 2  # the key cache one F layer scans
+    abytes = B * TOPK * HKV * 2 * DH * 2
+    del layers
+    torch.cuda.empty_cache()
+    return {"workload": f"decode B={B} at a {Lc}-token cache, 4 layers {pat}, H_I={H_I} d_I={D_I} top-{TOPK}, "
+                        f"GQA {HQ}Q/{HKV}KV d={DH}",
+            "tok_per_s": round(B / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "indexer_ms": round(idx_ms, 4), "attention_ms": round(att_ms, 4),
+            "indexer_gbs": round(kbytes / (idx_ms / 1e3) / 1e9, 1),
+            "attention_gathered_gbs": round(4 * abytes / (att_ms / 1e3) / 1e9, 1),
+            "all_f_ms_per_step": round(res["FFFF"][0], 4),
+            "all_f_tok_per_s": round(B / (res["FFFF"][0] / 1e3), 1)}
+
+
+def run_ctx1m(args, dev):
+    """The last 8192-token chunk of a 1M-token chunked prefill: fp8 indexer (H_I=64, d_I=128,
+    per-token scales) on 2 of 8 layers (FSSSFSSS), latent attention (576-dim rows, 512-dim values,
+    64 query heads) on all 8, against the full 1048576-token caches."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    L1, C, H1, HQ1 = 1 << 20, 8192, 64, 64
+    p0 = L1 - C
+    gen = synth.StructuredIndexer("ctx1m", 1, L1, H1, D_I, r=32, base_std=1.0, noise_std=0.2, device=dev, seed=3000)
+    layers = []
+    for l in range(N_LAYERS):
+        Lh = {}
+        if PATTERN[l] == "F":
+            q, w = gen.queries(l, p0, L1)
+            Lh["q_I"], Lh["q_scale"] = synth.quantize_e4m3_rows(q)
+            Lh["k_I"], Lh["k_scale"] = synth.quantize_e4m3_rows(gen.keys(l))
+            Lh["w"] = w
+        Lh["Q"], Lh["K"], _ = synth.attention_inputs("ctx1m", l, 1, C, L1, HQ1, 1, 576, None, device=dev, seed=3000)
+        Lh["O"] = torch.empty((1, C, HQ1, 512), dtype=torch.bfloat16, device=dev)
+        layers.append(Lh)
+    del gen
+    shape = dsa.group_shape(1, C, p0, L1, H1, D_I, HQ1, 1, 576, 512, TOPK, idx_dtype=dsa.DSA_E4M3,
+                            o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((1, C, TOPK), dtype=torch.int32, device=dev))
+    dsa.layer_group_forward(shape, layers, PATTERN, cache, workspace=ws)
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * N_LAYERS)]
+    for e in evs:
+        e.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    dsa.layer_group_forward(shape, layers, PATTERN, cache, workspace=ws, events=evs)
+    t1.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = t0.elapsed_time(t1)
+    idx_ms = [evs[3 * l].elapsed_time(evs[3 * l + 1]) for l in range(N_LAYERS) if PATTERN[l] == "F"]
+    att_ms = [evs[3 * l + 1].elapsed_time(evs[3 * l + 2]) for l in range(N_LAYERS)]
+    iflops = 2 * H1 * D_I * sum(range(p0 + 1, L1 + 1))
+    abytes = C * TOPK * 576 * 2
+    del layers
+    torch.cuda.empty_cache()
+    # whole 1M prefill estimate: indexer work grows with the chunk's position, attention does not
+    n_chunks = L1 // C
+    idx_avg = sum(idx_ms) / len(idx_ms)
+    est_s = (sum(att_ms) * n_chunks + idx_avg * 2 * sum((c * C + C / 2) / (p0 + C / 2) for c in range(n_chunks))) / 1e3
+    return {"workload": f"last {C}-token chunk of a {L1}-token chunked prefill, 8 layers {PATTERN}, fp8 e4m3 "
+                        f"indexer H_I={H1} d_I={D_I} top-{TOPK}, latent attention 576/512 with {HQ1} heads",
+            "chunk_ms": round(ms, 3), "chunk_tok_per_s": round(C / (ms / 1e3), 1),
+            "indexer_ms_per_f_layer": round(idx_avg, 3),
+            "indexer_fp8_tflops": round(iflops / (idx_avg / 1e3) / 1e12, 1),
+            "attention_ms_per_layer": round(sum(att_ms) / len(att_ms), 3),
+            "attention_gathered_gbs": round(abytes / (sum(att_ms) / len(att_ms) / 1e3) / 1e9, 1),
+            "full_prefill_estimate_s": round(est_s, 2),
+            "full_prefill_estimate_tok_per_s": round(L1 / est_s, 1)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,6 +547,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=24)
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench", choices=["bench", "profile"],
                     help="profile: small single-kernel launches for ncu captures")
     args = ap.parse_args()
@@ -459,6 +577,13 @@ def main():
         v, total, sample, threads, meas = oracle_sample(layers, args.cpu_rows)
         out["cpu_baseline"] = {"value": round(v, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
                                "sample": sample}
+    del layers
+    if not args.no_extra:
+        import torch
+        torch.cuda.empty_cache()
+        dev = torch.device("cuda", local_rank)
+        out["decode"] = run_decode(args, dev)
+        out["context_1m_tail_chunk"] = run_ctx1m(args, dev)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

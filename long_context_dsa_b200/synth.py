@@ -60,31 +60,46 @@ class StructuredIndexer:
     """Per-layer indexer inputs with a shared low-rank token structure.
 
     ``layer(l)`` returns (q_I [B, L, H, d] bf16, k_I [B, L, d] bf16, w [B, L, H] fp32).
-    The shared bases are built once per instance (fp32, on ``device``).
+    ``keys(l)`` returns that layer's k_I alone (the same values); ``queries(l, t0, t1)``
+    draws the query rows t0..t1-1 of the same recipe without building the full
+    query tensor (its noise is its own draw, so it is not a slice of ``layer``'s q_I).
+    The shared factors are built once per instance (fp32, on ``device``).
     """
 
     def __init__(self, name: str, B: int, L: int, H: int, d: int, r: int,
                  base_std: float, noise_std: float, device="cpu", seed: int = 0):
         self.name, self.B, self.L, self.H, self.d = name, B, L, H, d
         self.noise_std, self.device, self.seed = noise_std, device, seed
-        z = normal((B, L, r), seed_for(seed, name, "Z"), device)
-        a_q = normal((H, r, d), seed_for(seed, name, "A_q"), device, std=base_std / r ** 0.5)
+        self.z = normal((B, L, r), seed_for(seed, name, "Z"), device)
+        self.a_q = normal((H, r, d), seed_for(seed, name, "A_q"), device, std=base_std / r ** 0.5)
         a_k = normal((r, d), seed_for(seed, name, "A_k"), device, std=base_std / r ** 0.5)
-        # base_q[b,t,h,:] = Z[b,t] @ A_q[h]
-        self.base_q = torch.einsum("btr,hrd->bthd", z, a_q).contiguous()
-        self.base_k = (z @ a_k).contiguous()
+        self.base_k = (self.z @ a_k).contiguous()
         self.w = uniform((B, L, H), seed_for(seed, name, "w"), device)
-        del z
+
+    def _base_q(self, t0: int, t1: int) -> torch.Tensor:
+        # base_q[b,t,h,:] = Z[b,t] @ A_q[h]
+        return torch.einsum("btr,hrd->bthd", self.z[:, t0:t1], self.a_q).contiguous()
 
     def layer(self, l: int):
         B, L, H, d = self.B, self.L, self.H, self.d
         q = normal((B, L, H, d), seed_for(self.seed, self.name, l, "q_noise"), self.device, std=self.noise_std)
-        q.add_(self.base_q)
+        q.add_(self._base_q(0, L))
         q = q.to(torch.bfloat16)
+        return q, self.keys(l), self.w
+
+    def keys(self, l: int) -> torch.Tensor:
+        B, L, d = self.B, self.L, self.d
         k = normal((B, L, d), seed_for(self.seed, self.name, l, "k_noise"), self.device, std=self.noise_std)
         k.add_(self.base_k)
-        k = k.to(torch.bfloat16)
-        return q, k, self.w
+        return k.to(torch.bfloat16)
+
+    def queries(self, l: int, t0: int, t1: int):
+        """(q_I [B, t1-t0, H, d] bf16, w [B, t1-t0, H] fp32) for positions t0..t1-1."""
+        B, H, d = self.B, self.H, self.d
+        q = normal((B, t1 - t0, H, d), seed_for(self.seed, self.name, l, "q_rows", t0, t1), self.device,
+                   std=self.noise_std)
+        q.add_(self._base_q(t0, t1))
+        return q.to(torch.bfloat16), self.w[:, t0:t1].contiguous()
 
 
 def attention_inputs(name: str, l: int, B: int, L_q: int, L_kv: int, Hq: int, Hkv: int,
