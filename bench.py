@@ -548,11 +548,18 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
-    ap.add_argument("--case", default="bench", choices=["bench", "profile"],
-                    help="profile: small single-kernel launches for ncu captures")
+    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "ctx1m"],
+                    help="profile: small single-kernel launches for ncu captures; decode / ctx1m: only that "
+                         "extra measurement, printed as one JSON line")
     args = ap.parse_args()
     if args.case == "profile":
         run_profile_case(args)
+        return
+    if args.case in ("decode", "ctx1m"):
+        import torch
+        dev = torch.device("cuda", 0)
+        fn = run_decode if args.case == "decode" else run_ctx1m
+        print(json.dumps({"case": args.case, **fn(args, dev)}), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

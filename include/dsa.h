@@ -188,6 +188,10 @@ DSA_API int idx_cache_get(const dsa_index_cache* cache, int layer, const char* p
  *   O   [B, n_q, Hq, d_v]   fp32 (o_dtype DSA_F32) or bf16 (DSA_BF16)
  * Supported: d_qk == d_v in {64, 128} with Hq/Hkv in {1,2,4,8};
  * latent d_qk = 576, d_v = 512, Hkv = 1, Hq a multiple of 8.
+ * Workspace: the status word, plus (when B*n_q*Hkv is too small to occupy
+ * every warp of the GPU, e.g. decode) fp32 partial softmax state for each
+ * query head and range of the index list, merged by a second kernel.  The
+ * size depends on the shape and the device's SM count only.
  * ====================================================================== */
 DSA_API int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, int d_qk, int d_v,
                                     int topk, size_t* bytes);

@@ -23,6 +23,7 @@ cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* 
                                       int num_sms, cudaStream_t stream);
 size_t indexer_workspace_bytes(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype,
                                int num_sms);
+size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms);
 cudaError_t launch_indexer(const void* q, const float* q_scale, const void* k, const float* k_scale,
                            const float* w, int dtype, int B, int n_q, int q_pos0, int n_kv, int H, int d,
                            int topk, int* idx_out, float* scores_out, void* ws, size_t ws_bytes, int num_sms,
@@ -274,7 +275,14 @@ int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, i
     if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
     if (B < 1 || n_q < 1 || n_kv < 1 || Hq < 1 || Hkv < 1 || d_qk < 1 || d_v < 1 || topk < 1)
         return fail(DSA_ERR_INVALID_ARG, "bad sizes");
-    *bytes = kWsHeaderBytes;
+    size_t part = 0;
+    if (d_qk == d_v && Hkv > 0 && Hq % Hkv == 0) {
+        int sms;
+        int rc = sm_count(&sms);
+        if (rc) return rc;
+        part = sparse_attn_part_bytes(B, n_q, Hq, Hkv, d_qk, topk, sms);
+    }
+    *bytes = kWsHeaderBytes + part;
     return DSA_OK;
 }
 

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(WARPS * 32)
     sparse_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                        const __nv_bfloat16* __restrict__ V, const int* __restrict__ idx, int B, int n_q,
                        int n_kv, int Hq, int Hkv, int topk, float scale_log2, void* __restrict__ O,
-                       WsHeader* hdr) {
+                       int splits, int chunks_per_split, float* __restrict__ part, WsHeader* hdr) {
     using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,7 +99,10 @@ __global__ void __launch_bounds__(WARPS * 32)
     const uint32_t ring_s = smem_u32(ring);
 
     const int G = Hq / Hkv;
+    // work items: (query row, KV head) units, each cut into `splits` ranges of chunks; with
+    // splits > 1 a warp writes its range's softmax state to `part` and attn_merge_kernel combines
     const long long units = static_cast<long long>(B) * n_q * Hkv;
+    const long long items = units * splits;
     const int nchunks = (topk + CHUNK - 1) / CHUNK;
     const size_t tok_stride = static_cast<size_t>(Hkv) * D;  // elements per token row of K / V
 
@@ -110,8 +113,12 @@ __global__ void __launch_bounds__(WARPS * 32)
     const int v_key_off = ((lq >= 2) ? 8 : 0) + lrow, v_d_off = (lq & 1) ? 8 : 0;  // V: trans A
     const int seg = lane % C::SEGS, sub = lane / C::SEGS;  // copy: segment within a row, row within an insn
 
-    for (long long u = static_cast<long long>(blockIdx.x) * WARPS + warp; u < units;
-         u += static_cast<long long>(gridDim.x) * WARPS) {
+    for (long long it = static_cast<long long>(blockIdx.x) * WARPS + warp; it < items;
+         it += static_cast<long long>(gridDim.x) * WARPS) {
+        const long long u = it / splits;
+        const int sp = static_cast<int>(it % splits);
+        const int c0 = sp * chunks_per_split;
+        const int c1 = min(nchunks, c0 + chunks_per_split);
         const long long row = u / Hkv;
         const int g = static_cast<int>(u % Hkv);
         const long long b = row / n_q;
@@ -131,8 +138,8 @@ __global__ void __launch_bounds__(WARPS * 32)
         };
         // gather chunk c's K and V slices into stage c % STAGES (always commits one group)
         auto issue = [&](int c, int tsel) {
-            if (c < nchunks) {
-                const int s = c % STAGES;
+            if (c < c1) {
+                const int s = (c - c0) % STAGES;
                 if (lane < CHUNK) sidx[s * CHUNK + lane] = tsel;
                 const uint32_t kst = ring_s + s * C::STAGE_BYTES;
                 const uint32_t vst = kst + CHUNK * C::RS;
@@ -168,15 +175,15 @@ __global__ void __launch_bounds__(WARPS * 32)
         // prologue: stages 0 .. STAGES-2 in flight, the next chunk's indices in a register
         __syncwarp();
 #pragma unroll
-        for (int c = 0; c < STAGES - 1; ++c) issue(c, load_idx(c));
-        int t_next = load_idx(STAGES - 1);
+        for (int c = 0; c < STAGES - 1; ++c) issue(c0 + c, load_idx(c0 + c));
+        int t_next = load_idx(c0 + STAGES - 1);
 
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = c0; c < c1; ++c) {
             issue(c + STAGES - 1, t_next);
             t_next = load_idx(c + STAGES);
             cp_async_wait<STAGES - 1>();
             __syncwarp();
-            const int s = c % STAGES;
+            const int s = (c - c0) % STAGES;
             const uint32_t kst = ring_s + s * C::STAGE_BYTES;
             const uint32_t vst = kst + CHUNK * C::RS;
             const int* si = sidx + s * CHUNK;
@@ -273,6 +280,33 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) lrun[j] += __shfl_xor_sync(0xffffffffu, lrun[j], off);
         }
+        if (splits > 1) {
+            // this range's state per head: unnormalised O, running max (log2 units), sum
+            float* pb = part + static_cast<size_t>(it) * G * (D + 2);
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+                const int d0 = dt * 16 + qn;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = hc + j;
+                    if (h < G) {
+                        pb[h * (D + 2) + d0] = o[dt][j];
+                        pb[h * (D + 2) + d0 + 8] = o[dt][2 + j];
+                    }
+                }
+            }
+            if (qn == 0) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = hc + j;
+                    if (h < G) {
+                        pb[h * (D + 2) + D] = mrun[j];
+                        pb[h * (D + 2) + D + 1] = lrun[j];
+                    }
+                }
+            }
+            continue;
+        }
         const float inv0 = lrun[0] > 0.f ? 1.f / lrun[0] : 0.f;
         const float inv1 = lrun[1] > 0.f ? 1.f / lrun[1] : 0.f;
 #pragma unroll
@@ -299,6 +333,58 @@ __global__ void __launch_bounds__(WARPS * 32)
     }
 }
 
+// Combine the split ranges of each (query row, KV head, query head):
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.
+template <bool OUT_BF16>
+__global__ void attn_merge_kernel(const float* __restrict__ part, int G, int D, int splits, int Hq, int Hkv,
+                                  void* __restrict__ O) {
+    const long long u = blockIdx.x;  // (row, g)
+    const int h = blockIdx.y;
+    const long long row = u / Hkv;
+    const int g = static_cast<int>(u % Hkv);
+    const float* p0 = part + (static_cast<size_t>(u) * splits * G + h) * (D + 2);
+    const size_t sstride = static_cast<size_t>(G) * (D + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, p0[s * sstride + D]);
+    float L = 0.f;
+    for (int s = 0; s < splits; ++s) {
+        const float m = p0[s * sstride + D];
+        L += (m == -INFINITY) ? 0.f : exp2f(m - M) * p0[s * sstride + D + 1];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float m = p0[s * sstride + D];
+            if (m != -INFINITY) acc += exp2f(m - M) * p0[s * sstride + d];
+        }
+        const size_t ob = (static_cast<size_t>(row) * Hq + g * G + h) * D + d;
+        if (OUT_BF16)
+            reinterpret_cast<__nv_bfloat16*>(O)[ob] = __float2bfloat16_rn(acc * inv);
+        else
+            reinterpret_cast<float*>(O)[ob] = acc * inv;
+    }
+}
+
+// Warps per CTA of the two dense configurations (one CTA per SM fits in shared memory).
+static constexpr int kAttnWarpsD128 = 14;
+static constexpr int kAttnWarpsD64 = 16;
+
+// Ranges per unit: 1 unless there are too few (row, KV head) units to give every warp of the
+// GPU two work items.  Depends only on the shape and SM count, so the workspace query and the
+// launch agree.
+static int attn_splits(long long units, int nchunks, int warps, int num_sms, int* per) {
+    const long long want = 2ll * num_sms * warps;
+    int s = 1;
+    if (units < want) {
+        s = static_cast<int>((want + units - 1) / units);
+        const int most = nchunks / 4 > 1 ? nchunks / 4 : 1;  // at least 4 chunks per range
+        if (s > most) s = most;
+    }
+    *per = (nchunks + s - 1) / s;
+    return (nchunks + *per - 1) / *per;
+}
+
 template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ = false, bool QK_SPLIT = false>
 static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                                  const int* idx, int B, int n_q, int n_kv, int Hq, int Hkv, int topk,
@@ -314,14 +400,36 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     const long long units = static_cast<long long>(B) * n_q * Hkv;
+    const int nchunks = (topk + CHUNK - 1) / CHUNK;
+    int per = nchunks;
+    const int splits = attn_splits(units, nchunks, WARPS, num_sms, &per);
     long long grid = static_cast<long long>(num_sms) * per_sm;
-    const long long need = (units + WARPS - 1) / WARPS;
+    const long long need = (units * splits + WARPS - 1) / WARPS;
     if (grid > need) grid = need;
     if (grid < 1) grid = 1;
     const float scale_log2 = scale * 1.4426950408889634f;
+    float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(hdr) + kWsHeaderBytes);
     kern<<<static_cast<int>(grid), WARPS * 32, C::SMEM, stream>>>(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, topk,
-                                                                   scale_log2, O, hdr);
+                                                                   scale_log2, O, splits, per, part, hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    const int G = Hq / Hkv;
+    dim3 mg(static_cast<unsigned>(units), static_cast<unsigned>(G));
+    if (out_bf16)
+        attn_merge_kernel<true><<<mg, 128, 0, stream>>>(part, G, D, splits, Hq, Hkv, O);
+    else
+        attn_merge_kernel<false><<<mg, 128, 0, stream>>>(part, G, D, splits, Hq, Hkv, O);
     return cudaGetLastError();
+}
+
+// Bytes of split-range state the sparse attention needs beyond the status word.
+size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms) {
+    if (d != 128 && d != 64) return 0;
+    const int warps = d == 128 ? kAttnWarpsD128 : kAttnWarpsD64;
+    const long long units = static_cast<long long>(B) * n_q * Hkv;
+    int per = 0;
+    const int splits = attn_splits(units, (topk + 15) / 16, warps, num_sms, &per);
+    if (splits == 1) return 0;
+    return static_cast<size_t>(units) * splits * (Hq / Hkv) * (d + 2) * sizeof(float);
 }
 
 // Host dispatcher: returns cudaErrorNotSupported for shapes without a kernel.
@@ -334,10 +442,10 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
     // 16-key chunks, 2 stages per warp, swizzled rows: as many warps per SM as shared memory
     // holds (measured on B200: warps in flight matter more than stages per warp).
     if (d == 128)
-        return launch_attn_t<128, 16, 2, 14, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
+        return launch_attn_t<128, 16, 2, kAttnWarpsD128, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
                                                          out_bf16, hdr, num_sms, stream);
     if (d == 64)
-        return launch_attn_t<64, 16, 2, 16, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
+        return launch_attn_t<64, 16, 2, kAttnWarpsD64, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
                                                         out_bf16, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }

@@ -251,6 +251,12 @@ def idx_cache_get(cache: IndexCache, layer: int, pattern: str) -> torch.Tensor:
 
 
 # --------------------------------------------------------- sparse attention
+def sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk, ctypes.byref(n)))
+    return n.value
+
+
 def sparse_attn_topk(Q, K, V, idx, scale: float | None = None, o_dtype=torch.float32, d_v: int | None = None,
                      out=None, workspace=None, stream=None) -> torch.Tensor:
     """O[b,i,h] = softmax over idx[b,i] of scale*Q.K, times V -> [B, n_q, Hq, d_v]."""
@@ -271,9 +277,7 @@ def sparse_attn_topk(Q, K, V, idx, scale: float | None = None, o_dtype=torch.flo
         out = torch.empty((B, n_q, Hq, d_v), dtype=o_dtype, device=Q.device)
     _need(out, o_dtype, "out")
     if workspace is None:
-        n = ctypes.c_size_t(0)
-        _check(lib().sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk, ctypes.byref(n)))
-        workspace = _workspace(n.value, Q.device)
+        workspace = _workspace(sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk), Q.device)
     _check(lib().sparse_attn_topk(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk,
                                   float(scale or 0.0), _ptr(out), od, _ptr(workspace), workspace.numel(),
                                   _stream(stream)))

@@ -32,6 +32,10 @@ CASES = [
     ("gqa8x1_d128", 1, 200, 0, 200, 8, 1, 128, 50, None),
     ("gqa4x4_d64", 1, 300, 0, 300, 4, 4, 64, 33, None),
     ("decode_b4", 4, 1, 4999, 5000, 32, 4, 128, 2048, None),
+    ("decode_b64_d64", 64, 1, 2999, 3000, 16, 2, 64, 1000, None),
+    ("decode_b16_mha8", 16, 1, 1999, 2000, 8, 8, 128, 2000, None),
+    ("decode_b3_k37", 3, 1, 99, 100, 32, 4, 128, 37, None),
+    ("chunk4_b8_k2048", 8, 4, 2996, 3000, 32, 4, 128, 2048, None),
     ("chunk_b2", 2, 100, 900, 1000, 32, 4, 128, 300, None),
 ]
 
@@ -41,7 +45,8 @@ def test_sparse_attention_matches_oracle(case):
     name, B, n_q, q_pos0, n_kv, Hq, Hkv, d, k, sample = case
     Q, K, V = synth.attention_inputs(name, 0, B, n_q, n_kv, Hq, Hkv, d, d)
     idx = _indices(n_kv, k, 1, q_pos0, n_q, B)
-    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(dsa.sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d, d, k), dtype=torch.uint8,
+                     device=DEV)
     O = dsa.sparse_attn_topk(Q.to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV), workspace=ws)
     assert dsa.read_status(ws) == 0
     O = O.cpu().numpy()
@@ -86,13 +91,32 @@ def test_out_of_range_index_is_skipped_and_flagged():
     idx = _indices(L, k, 6)
     idx[0, 10, 0] = L + 5      # beyond the cache
     idx[0, 11, 1] = -7         # negative, not the -1 pad
-    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(dsa.sparse_attn_topk_workspace_size(1, L, L, Hq, Hkv, d, d, k), dtype=torch.uint8, device=DEV)
     O = dsa.sparse_attn_topk(Q.to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV), workspace=ws)
     assert dsa.read_status(ws) & dsa.STATUS_BAD_INDEX
     clean = idx.copy()
     clean[0, 10, 0] = -1
     clean[0, 11, 1] = -1
     check_attention(O.cpu().numpy()[0], oracle.sparse_attention(Q[0], K[0], V[0], clean[0]))
+
+
+def test_split_ranges_decode_flags_bad_index_and_merges():
+    """Few rows -> the index list is cut into ranges merged afterwards; padding-only ranges stay neutral."""
+    B, L, Hq, Hkv, d, k = 2, 3000, 32, 4, 128, 2048
+    Q, K, V = synth.attention_inputs("split", 0, B, 1, L, Hq, Hkv, d, d)
+    idx = _indices(L, k, 12, L - 1, 1, B)
+    idx[0, 0, 700:1500] = -1     # whole ranges of padding in the middle
+    idx[1, 0, 5] = L + 3
+    need = dsa.sparse_attn_topk_workspace_size(B, 1, L, Hq, Hkv, d, d, k)
+    assert need > 256            # split-range state is in use for this shape
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    O = dsa.sparse_attn_topk(Q.to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV), workspace=ws)
+    assert dsa.read_status(ws) & dsa.STATUS_BAD_INDEX
+    clean = idx.copy()
+    clean[1, 0, 5] = -1
+    O = O.cpu().numpy()
+    for b in range(B):
+        check_attention(O[b], oracle.sparse_attention(Q[b], K[b], V[b], clean[b]))
 
 
 def test_bf16_output():
