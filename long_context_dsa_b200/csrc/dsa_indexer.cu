@@ -242,6 +242,7 @@ __global__ void __launch_bounds__(320, 1)
         constexpr int CHECK = 4;                       // prune checks every CHECK key tiles
         const int sub = grp.sub();                     // this warp's share of a row buffer
         const int room = sub - CHECK * 32;             // prune once a sub-buffer holds more than this
+        const int slack = max(32, p.topk / 8);         // a prune may keep up to k + slack candidates
         uint32_t u = 0;
         bool ok = true;
         for (int r = 0; ok; ++r) {
@@ -387,7 +388,8 @@ __global__ void __launch_bounds__(320, 1)
                         for (int q = 0; q < C::QG; ++q) {
                             if ((need >> q) & 1ull) {
                                 uint32_t* ck = cbase + static_cast<size_t>(q) * 2 * p.cap;
-                                grp.prune(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk, room - 32, sortbuf);
+                                grp.prune_fast(&st[q], ck, reinterpret_cast<int*>(ck + p.cap), p.topk, room - 32,
+                                               slack, sortbuf);
                             }
                         }
 #pragma unroll

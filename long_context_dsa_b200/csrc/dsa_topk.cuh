@@ -112,6 +112,47 @@ struct TopkGroup {
         return r;
     }
 
+    // Over the summed per-warp histograms of 256 bins: the bin holding the
+    // kk-th largest item (sel_digit), the count above it (sel_above) and in it
+    // (sel_equal).  Threads 0-31 work; the caller syncs before and after.
+    __device__ void scan_bins(int kk) const {
+        if (tid < 32) {
+            const int lane = tid;
+            int cnt8[8];
+            int s8 = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                int c = 0;
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww) c += sc->hist[ww][lane * 8 + j];
+                cnt8[j] = c;
+                s8 += c;
+            }
+            int suf = s8;  // count in bins >= lane*8
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_down_sync(0xffffffffu, suf, off);
+                if (lane + off < 32) suf += o;
+            }
+            const unsigned ball = __ballot_sync(0xffffffffu, suf >= kk);
+            const int L = 31 - __clz(ball);
+            if (lane == L) {
+                int acc = suf - s8;
+                bool found = false;
+#pragma unroll
+                for (int j = 7; j >= 0; --j) {
+                    if (!found && acc + cnt8[j] >= kk) {
+                        sc->sel_digit = L * 8 + j;
+                        sc->sel_above = acc;
+                        sc->sel_equal = cnt8[j];
+                        found = true;
+                    }
+                    acc += cnt8[j];
+                }
+            }
+        }
+    }
+
     // kk-th largest (1-based, kk <= number of participants) of the
     // participating items v[i] (bit i of `part`) over the whole group.
     // n_greater / n_equal count the participants above / equal to it.
@@ -151,41 +192,7 @@ struct TopkGroup {
                 if (((part >> i) & 1u) && (v[i] & fixed) == prefix) atomicAdd(&sc->hist[w][(v[i] >> shift) & dmask], 1);
             }
             sync();
-            if (tid < 32) {
-                const int lane = tid;
-                int cnt8[8];
-                int s8 = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    int c = 0;
-#pragma unroll
-                    for (int ww = 0; ww < NW; ++ww) c += sc->hist[ww][lane * 8 + j];
-                    cnt8[j] = c;
-                    s8 += c;
-                }
-                int suf = s8;  // count in bins >= lane*8
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int o = __shfl_down_sync(0xffffffffu, suf, off);
-                    if (lane + off < 32) suf += o;
-                }
-                const unsigned ball = __ballot_sync(0xffffffffu, suf >= kk);
-                const int L = 31 - __clz(ball);
-                if (lane == L) {
-                    int acc = suf - s8;
-                    bool found = false;
-#pragma unroll
-                    for (int j = 7; j >= 0; --j) {
-                        if (!found && acc + cnt8[j] >= kk) {
-                            sc->sel_digit = L * 8 + j;
-                            sc->sel_above = acc;
-                            sc->sel_equal = cnt8[j];
-                            found = true;
-                        }
-                        acc += cnt8[j];
-                    }
-                }
-            }
+            scan_bins(kk);
             sync();
             const int dsel = sc->sel_digit;
             kk -= sc->sel_above;
@@ -364,6 +371,111 @@ struct TopkGroup {
 #pragma unroll
             for (int ww = 0; ww < NW; ++ww) st->cnt[ww] = max(0, min(qn, total - ww * qn));
         }
+        sync();
+    }
+
+    // Streaming prune: keeps, in place and in order, every candidate whose key
+    // is at least a threshold T chosen so that at least k and at most
+    // k + slack candidates qualify -- a superset of the row's current top k,
+    // so nothing that can still be selected is dropped -- and raises the
+    // admission threshold to T (ties at T are admitted).  T is the lower edge
+    // of the bin that holds the k-th key in a 256-bin histogram over the key
+    // range [current threshold, largest key], refined inside that bin until
+    // it is small enough; usually one pass against the several digit passes
+    // of an exact select.  Falls back to the exact prune when one key value
+    // carries more ties than the slack, or when one warp would keep more than
+    // keep_max.  Same calling rules as prune.
+    __device__ void prune_fast(TopkRowState* st, uint32_t* ckey, int* cidx, int k, int keep_max, int slack,
+                               int* sortbuf) const {
+        int total0 = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) total0 += min(st->cnt[w], sub());
+        if (total0 <= k) return;
+        uint32_t rk[PER];
+        int ri[PER];
+        uint32_t valid;
+        load_own(st, ckey, cidx, rk, ri, valid);
+        uint32_t lo = st->thr_key;  // every candidate's key is at least the threshold it passed
+        uint32_t hi = 0u, lo_inv = 0u;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            if ((valid >> i) & 1u) {
+                hi = max(hi, rk[i]);
+                lo_inv = max(lo_inv, ~rk[i]);
+            }
+        }
+        hi = umax_reduce(hi);
+        if (lo == 0u) lo = ~umax_reduce(lo_inv);  // first prune of the row (uniform: lo is shared)
+        const int w = warp(), lane = tid & 31, s_ = sub();
+        int above = 0, kk = k;
+        uint32_t T = lo;
+        bool exact = false;
+#pragma unroll 1
+        while (true) {
+            const uint32_t span = hi - lo;
+            const int sh = span < 256u ? 0 : (32 - __clz(span)) - 8;  // bins of 2^sh keys
+            for (int b = tid; b < NW * 256; b += NT) (&sc->hist[0][0])[b] = 0;
+            sync();
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                if (((valid >> i) & 1u) && rk[i] >= lo && rk[i] <= hi) atomicAdd(&sc->hist[w][(rk[i] - lo) >> sh], 1);
+            }
+            sync();
+            scan_bins(kk);
+            sync();
+            const uint32_t blo = lo + (static_cast<uint32_t>(sc->sel_digit) << sh);
+            const int ab = sc->sel_above, eqc = sc->sel_equal;
+            above += ab;
+            kk -= ab;
+            if (above + eqc <= k + slack) {  // keep the whole bin
+                T = blo;
+                break;
+            }
+            if (sh == 0) {  // one key value with more ties than the slack
+                exact = true;
+                break;
+            }
+            const uint32_t wmask = (1u << sh) - 1u;
+            hi = (hi - blo > wmask) ? blo + wmask : hi;
+            lo = blo;
+        }
+        if (exact) {
+            prune(st, ckey, cidx, k, keep_max, sortbuf);
+            return;
+        }
+        uint32_t keep = 0u;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) keep |= ((((valid >> i) & 1u) && rk[i] >= T) ? 1u : 0u) << i;
+        const unsigned lt = (1u << lane) - 1u;
+        int wkeep = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) wkeep += __popc(__ballot_sync(0xffffffffu, (keep >> i) & 1u));
+        if (lane == 0) sc->warp_val[w] = wkeep;
+        sync();  // every load above is done before any store below
+        int wmax = 0;
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) wmax = max(wmax, sc->warp_val[ww]);
+        sync();
+        if (wmax > keep_max) {
+            prune(st, ckey, cidx, k, keep_max, sortbuf);
+            return;
+        }
+        int b = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const unsigned m = __ballot_sync(0xffffffffu, (keep >> i) & 1u);
+            if ((keep >> i) & 1u) {
+                const int pos = b + __popc(m & lt);
+                ckey[w * s_ + pos] = rk[i];
+                cidx[w * s_ + pos] = ri[i];
+            }
+            b += __popc(m);
+        }
+        if (tid == 0) {
+            st->thr_key = T;
+            st->thr_idx = 0x7fffffff;
+        }
+        if (lane == 0) st->cnt[w] = wkeep;
         sync();
     }
 
