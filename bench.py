@@ -109,17 +109,14 @@ class ClockSampler:
 # ------------------------------------------------------------- GPU arm
 def run_gpu(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
-    from long_context_dsa_b200 import dsa, synth
+    from long_context_dsa_b200 import dsa, replicas
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     hbm, bf16_burst, bf16_sus, peak_src = peaks()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = replicas.barrier
 
     # ---- inputs (seeded; each rank its own sequence)
     layers = make_layers(dev, rank)
@@ -183,18 +180,14 @@ def run_gpu(args, rank, world, local_rank):
     # ---- end to end through the public API from pinned host memory
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, layers, shape, cache, ws, dev, stream)
+        e2e = run_e2e(args, layers, shape, cache, ws, dev, stream, world)
 
     # ---- max over ranks
-    ms = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = replicas.max_over_ranks(ms_local, dev)
     ms_per_step = ms / args.steps
     idx_avg = sum(idx_ms) / len(idx_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
-    value = world * L / (ms_per_step / 1e3)
+    value = replicas.job_throughput(L, world, ms_per_step)
 
     abytes = attn_bytes()
     iflops = indexer_flops()
@@ -238,11 +231,11 @@ def run_gpu(args, rank, world, local_rank):
     return out, layers
 
 
-def run_e2e(args, layers, shape, cache, ws, dev, stream):
+def run_e2e(args, layers, shape, cache, ws, dev, stream, world=1):
     """Same metric through layer_group_forward with host buffers: every step copies its inputs
     host->device from pinned memory and reads every layer's output back."""
     import torch
-    from long_context_dsa_b200 import dsa
+    from long_context_dsa_b200 import dsa, replicas
 
     names_f = ("q_I", "k_I", "w", "Q", "K", "V")
     names_s = ("Q", "K", "V")
@@ -268,14 +261,15 @@ def run_e2e(args, layers, shape, cache, ws, dev, stream):
     one()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replicas.barrier()
     a.record(stream)
     for _ in range(steps):
         one()
     b.record(stream)
     torch.cuda.synchronize()
     dsa.check_status(ws)
-    ms = a.elapsed_time(b) / steps
-    return {"value": round(L / (ms / 1e3), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+    ms = replicas.max_over_ranks(a.elapsed_time(b) / steps, dev)
+    return {"value": round(replicas.job_throughput(L, world, ms), 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms, 3),
             "note": "pinned host inputs copied in and every layer's bf16 output read back inside the timed region"}
 
@@ -286,15 +280,18 @@ def make_layers(dev, rank=0, keep_indexer_all=True):
     import torch
     from long_context_dsa_b200 import synth
 
+    from long_context_dsa_b200 import replicas
+
+    seed = replicas.rank_seed(1000, rank)
     gen = synth.StructuredIndexer("prefill200k", 1, L, H_I, D_I, r=32, base_std=1.0, noise_std=0.2,
-                                  device=dev, seed=1000 + rank)
+                                  device=dev, seed=seed)
     layers = []
     for l in range(N_LAYERS):
         Lh = {}
         if keep_indexer_all or PATTERN[l] == "F":
             Lh["q_I"], Lh["k_I"], Lh["w"] = gen.layer(l)
         Lh["Q"], Lh["K"], Lh["V"] = synth.attention_inputs("prefill200k", l, 1, L, L, HQ, HKV, DH, DH,
-                                                           device=dev, seed=1000 + rank)
+                                                           device=dev, seed=seed)
         layers.append(Lh)
     del gen
     return layers
