@@ -57,7 +57,8 @@ struct IdxCfg {
     static constexpr int OFF_BAR = OFF_SORT + 2 * DSA_TOPK_MAX * 4;
     static constexpr int NBAR = 2 + 2 * STAGES + 4;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+    static constexpr int OFF_NEED = OFF_MISC + 16;  // [2 parities][2 groups][need, soft] prune masks
+    static constexpr int SMEM = OFF_NEED + 64 + 1024;  // + alignment slack
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     static_assert(D * ESZ % 128 == 0, "rows must be whole 128-byte swizzle blocks");
 };
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
     int* wg_abort = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);  // [2], written only by each group
+    unsigned long long* sNeed = reinterpret_cast<unsigned long long*>(smem + C::OFF_NEED);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
@@ -243,6 +245,9 @@ __global__ void __launch_bounds__(320, 1)
         const int sub = grp.sub();                     // this warp's share of a row buffer
         const int room = sub - CHECK * 32;             // prune once a sub-buffer holds more than this
         const int slack = max(32, p.topk / 8);         // a prune may keep up to k + slack candidates
+        // a row past this fill is pruned early when the other group stalls the MMA for a prune anyway
+        const int soft_room = (room + (p.topk + slack) / 4) / 2;
+        uint32_t chk = 0;                              // check points passed (same count in both groups)
         uint32_t u = 0;
         bool ok = true;
         for (int r = 0; ok; ++r) {
@@ -368,7 +373,7 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     grp.sync();
                     // decisions every thread of the group takes alike (read between two barriers)
-                    unsigned long long need = 0ull;
+                    unsigned long long need = 0ull, soft = 0ull;
 #pragma unroll
                     for (int q = 0; q < C::QG; ++q) {
                         int mx = 0, tot = 0;
@@ -378,10 +383,20 @@ __global__ void __launch_bounds__(320, 1)
                             tot += st[q].cnt[ww];
                         }
                         need |= (mx > room && tot > p.topk) ? (1ull << q) : 0ull;
+                        soft |= (mx > soft_room && tot > p.topk) ? (1ull << q) : 0ull;
                         if (mx > sub && tid == 0) raise_status(p.hdr, DSA_STATUS_OVERFLOW, mx);
                     }
-                    const bool stop = wg_abort[g] != 0;
-                    grp.sync();
+                    // Both groups meet here at the same key tile.  A prune holds its group's
+                    // accumulator, and the MMA alternates between the two, so a prune in one group
+                    // stalls both: rows of the other group that are well on their way to a prune
+                    // are pruned in the same stall.  The barrier also orders every read of the
+                    // counts above before any prune below.
+                    unsigned long long* nb = sNeed + (chk & 1u) * 4;
+                    if (tid == 0) nb[2 * g] = need;
+                    named_bar_sync(3, 256);
+                    const bool stop = (wg_abort[0] | wg_abort[1]) != 0;
+                    if (nb[2 * (g ^ 1)] != 0ull) need |= soft;
+                    ++chk;
                     if (stop) { ok = false; break; }
                     if (!SCORES && need) {
 #pragma unroll 1
