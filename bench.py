@@ -107,6 +107,15 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
+def attn_traffic():
+    """DRAM bytes of one full sparse-attention launch, scaled from the ncu capture of the tail case
+    (4096 rows x 2048 selected keys: 2.558 GB read + 0.036 GB written) by selected (query, key) pairs;
+    an over-estimate (earlier rows hit L2 more).  Update with the capture when the kernel changes."""
+    per_pair = (2.558264e9 + 0.036444e9) / (4096 * 2048)
+    pairs = sum(min(TOPK, t + 1) for t in range(L))
+    return round(per_pair * pairs)
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     from long_context_dsa_b200 import dsa, replicas
@@ -205,7 +214,7 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {
             "bound": "hbm", "kernel": "sparse_attn_kernel (gathered K/V rows)",
             "achieved": round(abytes / (attn_avg / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(abytes / (attn_avg / 1e3) / 1e9 / hbm, 4), "traffic": None,
+            "frac": round(abytes / (attn_avg / 1e3) / 1e9 / hbm, 4), "traffic": attn_traffic(),
             "peak_source": f"{peak_src} hbm_gbs",
             "algorithmic_bytes_per_launch": abytes, "avg_launch_ms": round(attn_avg, 3)},
         "indexer_roofline": {
