@@ -485,6 +485,71 @@ def run_decode(args, dev):
             "all_f_tok_per_s": round(B / (res["FFFF"][0] / 1e3), 1)}
 
 
+def run_mtp(args, dev):
+    """Multi-token (speculative) decode: 64 sequences verify 4 draft tokens each at a 200000-token
+    cache, 4 layers FSSS.  Shared: the F layer selects once, for the last draft token, and all 4
+    tokens attend through that selection (each causally up to its own position).  Unshared: one
+    selection per token (4 indexer launches) and per-token attention."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    B, Lc, m, nl = 64, 200000, 4, 4
+    p0 = Lc - m
+    gen = synth.StructuredIndexer("mtp200k", B, Lc, H_I, D_I, r=32, base_std=1.0, noise_std=0.2, device=dev,
+                                  seed=3000)
+    q_all, w_all = gen.queries(0, p0, Lc)
+    k_I = gen.keys(0)
+    del gen
+    q_last, w_last = q_all[:, m - 1:].contiguous(), w_all[:, m - 1:].contiguous()
+    q_tok = [q_all[:, j:j + 1].contiguous() for j in range(m)]
+    w_tok = [w_all[:, j:j + 1].contiguous() for j in range(m)]
+    att = [synth.attention_inputs("mtp200k", l, B, m, Lc, HQ, HKV, DH, DH, device=dev, seed=3000) for l in range(nl)]
+    Q_tok = [[Q[:, j:j + 1].contiguous() for j in range(m)] for (Q, _, _) in att]
+    O = torch.empty((B, m, HQ, DH), dtype=torch.bfloat16, device=dev)
+    O1 = [torch.empty((B, 1, HQ, DH), dtype=torch.bfloat16, device=dev) for _ in range(m)]
+    idx_s = torch.empty((B, 1, TOPK), dtype=torch.int32, device=dev)
+    idx_u = [torch.empty((B, 1, TOPK), dtype=torch.int32, device=dev) for _ in range(m)]
+    need = [dsa.idx_score_topk_workspace_size(B, 1, p0 + j, Lc, H_I, D_I, TOPK) for j in range(m)]
+    need += [dsa.sparse_attn_topk_workspace_size(B, n, Lc, HQ, HKV, DH, DH, TOPK) for n in (1, m)]
+    ws = torch.zeros(max(need), dtype=torch.uint8, device=dev)
+
+    def shared():
+        dsa.idx_score_topk(q_last, k_I, w_last, TOPK, q_pos0=Lc - 1, out=idx_s, workspace=ws)
+        for (Q, K, V) in att:
+            dsa.sparse_attn_topk_shared(Q, K, V, idx_s, m, p0, o_dtype=torch.bfloat16, out=O, workspace=ws)
+
+    def unshared():
+        for j in range(m):
+            dsa.idx_score_topk(q_tok[j], k_I, w_tok[j], TOPK, q_pos0=p0 + j, out=idx_u[j], workspace=ws)
+        for l, (Q, K, V) in enumerate(att):
+            for j in range(m):
+                dsa.sparse_attn_topk(Q_tok[l][j], K, V, idx_u[j], o_dtype=torch.bfloat16, out=O1[j], workspace=ws)
+
+    res = {}
+    for name, fn in (("shared", shared), ("unshared", unshared)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 10
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        dsa.check_status(ws)
+        res[name] = a.elapsed_time(b) / n
+    del att, Q_tok, k_I
+    torch.cuda.empty_cache()
+    return {"workload": f"multi-token decode: B={B} sequences verify {m} draft tokens at a {Lc}-token cache, "
+                        f"{nl} layers FSSS, H_I={H_I} d_I={D_I} top-{TOPK}, GQA {HQ}Q/{HKV}KV d={DH}",
+            "shared_ms_per_step": round(res["shared"], 4),
+            "shared_tok_per_s": round(B * m / (res["shared"] / 1e3), 1),
+            "unshared_ms_per_step": round(res["unshared"], 4),
+            "unshared_tok_per_s": round(B * m / (res["unshared"] / 1e3), 1),
+            "speedup": round(res["unshared"] / res["shared"], 3)}
+
+
 def run_ctx1m(args, dev):
     """The last 8192-token chunk of a 1M-token chunked prefill: fp8 indexer (H_I=64, d_I=128,
     per-token scales) on 2 of 8 layers (FSSSFSSS), latent attention (576-dim rows, 512-dim values,
@@ -554,17 +619,17 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
-    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "ctx1m"],
+    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "ctx1m", "mtp"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m: only that "
                          "extra measurement, printed as one JSON line")
     args = ap.parse_args()
     if args.case == "profile":
         run_profile_case(args)
         return
-    if args.case in ("decode", "ctx1m"):
+    if args.case in ("decode", "ctx1m", "mtp"):
         import torch
         dev = torch.device("cuda", 0)
-        fn = run_decode if args.case == "decode" else run_ctx1m
+        fn = {"decode": run_decode, "ctx1m": run_ctx1m, "mtp": run_mtp}[args.case]
         print(json.dumps({"case": args.case, **fn(args, dev)}), flush=True)
         return
 
@@ -596,6 +661,7 @@ def main():
         torch.cuda.empty_cache()
         dev = torch.device("cuda", local_rank)
         out["decode"] = run_decode(args, dev)
+        out["multi_token_decode"] = run_mtp(args, dev)
         out["context_1m_tail_chunk"] = run_ctx1m(args, dev)
     if world > 1:
         import torch.distributed as dist

@@ -200,6 +200,26 @@ DSA_API int sparse_attn_topk(const void* Q, const void* K, const void* V, const 
                      float scale, void* O, int o_dtype,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* sparse_attn_topk_shared -- the same attention where consecutive query rows
+ * share one index row (multi-token / speculative decode).
+ *
+ * [Term] §IndexShare: the sharing that lets layers reuse one indexer also
+ * raised MTP speculative-decoding acceptance; this entry point lets several
+ * query tokens of a sequence (a verified draft) reuse one F-layer selection.
+ * Query row i of sequence b (absolute position q_pos0 + i) uses index row
+ * idx[b, i / q_per_idx] and skips the entries of that row beyond its own
+ * position, so a selection made for the group's last token serves every
+ * token of the group causally.
+ *   idx [B, ceil(n_q / q_per_idx), topk] int32; everything else as in
+ *   sparse_attn_topk (workspace size from sparse_attn_topk_workspace_size
+ *   with the same B, n_q).  Requires q_per_idx >= 1 and
+ *   0 <= q_pos0, q_pos0 + n_q <= n_kv.
+ */
+DSA_API int sparse_attn_topk_shared(const void* Q, const void* K, const void* V, const int32_t* idx,
+                            int B, int n_q, int q_pos0, int n_kv, int Hq, int Hkv, int d_qk, int d_v,
+                            int topk, int q_per_idx, float scale, void* O, int o_dtype,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* ======================================================================
  * layer_group_forward -- one layer group: F layers index, S layers reuse.
  *

@@ -17,10 +17,10 @@ cudaError_t launch_topk_scores(const float* scores, int rows, int q_pos0, int n_
                                WsHeader* hdr, int num_sms, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, const int* idx, int B, int n_q,
                                int n_kv, int Hq, int Hkv, int d, int topk, float scale, void* O, bool out_bf16,
-                               WsHeader* hdr, int num_sms, cudaStream_t stream);
+                               IdxShare share, WsHeader* hdr, int num_sms, cudaStream_t stream);
 cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
-                                      int Hq, int topk, float scale, void* O, bool out_bf16, WsHeader* hdr,
-                                      int num_sms, cudaStream_t stream);
+                                      int Hq, int topk, float scale, void* O, bool out_bf16, IdxShare share,
+                                      WsHeader* hdr, int num_sms, cudaStream_t stream);
 size_t indexer_workspace_bytes(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype,
                                int num_sms);
 size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms);
@@ -286,9 +286,10 @@ int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, i
     return DSA_OK;
 }
 
-int sparse_attn_topk(const void* Q, const void* K, const void* V, const int32_t* idx, int B, int n_q, int n_kv,
-                     int Hq, int Hkv, int d_qk, int d_v, int topk, float scale, void* O, int o_dtype,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+int attn_common(const void* Q, const void* K, const void* V, const int32_t* idx, int B, int n_q, int n_kv, int Hq,
+                int Hkv, int d_qk, int d_v, int topk, float scale, void* O, int o_dtype, dsa::IdxShare share,
+                void* workspace, size_t workspace_bytes, void* stream) {
     int rc = check_attn_shape(V, B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk);
     if (rc) return rc;
     if (!Q || !K || !idx || !O) return fail(DSA_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -303,13 +304,33 @@ int sparse_attn_topk(const void* Q, const void* K, const void* V, const int32_t*
     if ((rc = sm_count(&sms))) return rc;
     cudaError_t e;
     if (V == nullptr)
-        e = launch_sparse_attn_latent(Q, K, idx, B, n_q, n_kv, Hq, topk, scale, O, o_dtype == DSA_BF16,
+        e = launch_sparse_attn_latent(Q, K, idx, B, n_q, n_kv, Hq, topk, scale, O, o_dtype == DSA_BF16, share,
                                       static_cast<WsHeader*>(workspace), sms, static_cast<cudaStream_t>(stream));
     else
         e = launch_sparse_attn(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, d_qk, topk, scale, O, o_dtype == DSA_BF16,
-                               static_cast<WsHeader*>(workspace), sms, static_cast<cudaStream_t>(stream));
+                               share, static_cast<WsHeader*>(workspace), sms, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "sparse_attn_topk");
     return DSA_OK;
+}
+}  // namespace
+
+int sparse_attn_topk(const void* Q, const void* K, const void* V, const int32_t* idx, int B, int n_q, int n_kv,
+                     int Hq, int Hkv, int d_qk, int d_v, int topk, float scale, void* O, int o_dtype,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+    return attn_common(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk, scale, O, o_dtype, dsa::kNoShare,
+                       workspace, workspace_bytes, stream);
+}
+
+int sparse_attn_topk_shared(const void* Q, const void* K, const void* V, const int32_t* idx, int B, int n_q,
+                            int q_pos0, int n_kv, int Hq, int Hkv, int d_qk, int d_v, int topk, int q_per_idx,
+                            float scale, void* O, int o_dtype, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    if (q_per_idx < 1) return fail(DSA_ERR_INVALID_ARG, "q_per_idx must be >= 1");
+    if (q_pos0 < 0 || static_cast<long long>(q_pos0) + n_q > n_kv)
+        return fail(DSA_ERR_INVALID_ARG, "query positions q_pos0..q_pos0+n_q-1 must lie inside the cache");
+    const dsa::IdxShare share = {q_per_idx, q_pos0, 1};
+    return attn_common(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk, scale, O, o_dtype, share, workspace,
+                       workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------- layer group

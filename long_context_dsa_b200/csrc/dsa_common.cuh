@@ -29,6 +29,18 @@ __device__ __forceinline__ void raise_status(WsHeader* h, int bits, int detail) 
     }
 }
 
+// Index rows shared by consecutive query rows (multi-token decode): query row i of
+// a sequence uses index row i / q_per_idx and skips entries after its own absolute
+// position q_pos0 + i.  q_per_idx = 1 without a position limit is the plain case.
+struct IdxShare {
+    int q_per_idx;
+    int q_pos0;    // absolute position of query row 0; ignored when causal == 0
+    int causal;
+    __host__ __device__ int rows(int n_q) const { return (n_q + q_per_idx - 1) / q_per_idx; }
+    __host__ __device__ int limit(int i) const { return causal ? q_pos0 + i : 0x7fffffff; }
+};
+static constexpr IdxShare kNoShare = {1, 0, 0};
+
 // Nanoseconds from the global timer.
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;

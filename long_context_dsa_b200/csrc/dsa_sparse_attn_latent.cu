@@ -74,7 +74,7 @@ template <int WARPS, bool OUT_BF16>
 __global__ void __launch_bounds__(WARPS * 32, 1)
     latent_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ KV,
                        const int* __restrict__ idx, int B, int n_q, int n_kv, int Hq, int topk, float scale_log2,
-                       void* __restrict__ O, WsHeader* hdr) {
+                       void* __restrict__ O, IdxShare share, WsHeader* hdr) {
     using C = Cfg<WARPS>;
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char* sq = smem;
@@ -98,7 +98,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         const long long row = u / hblocks;
         const int hb = static_cast<int>(u % hblocks);
         const long long b = row / n_q;
-        const int* irow = idx + row * topk;
+        const int qi = static_cast<int>(row - b * n_q);
+        const int* irow = idx + (b * share.rows(n_q) + qi / share.q_per_idx) * topk;
+        const int lim = share.limit(qi);  // shared rows: keys past this query's own position are skipped
         const __nv_bfloat16* kvb = KV + static_cast<size_t>(b) * n_kv * DQK;
 
         __syncthreads();  // the previous unit is done with the query block and the ring
@@ -120,13 +122,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                         raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
                         t = -1;
                     }
-                    sidx[s * CHUNK + threadIdx.x] = t;
+                    sidx[s * CHUNK + threadIdx.x] = t > lim ? -1 : t;
                 }
                 for (int sgi = threadIdx.x; sgi < CHUNK * SEGS; sgi += nthr) {
                     const int key = sgi / SEGS, sg = sgi % SEGS;
                     const int kk = c * CHUNK + key;
                     int t = kk < topk ? __ldg(irow + kk) : -1;
-                    const bool ok = t >= 0 && t < n_kv;
+                    const bool ok = t >= 0 && t < n_kv && t <= lim;
                     cp_async16(ring_s + s * C::STAGE_BYTES + key * RS + sg * 16,
                                kvb + static_cast<size_t>(ok ? t : 0) * DQK + sg * 8, ok ? 16u : 0u);
                 }
@@ -238,7 +240,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 
 template <int WARPS>
 cudaError_t launch_w(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv, int Hq, int topk,
-                     float scale, void* O, bool out_bf16, WsHeader* hdr, int num_sms, cudaStream_t stream) {
+                     float scale, void* O, bool out_bf16, IdxShare share, WsHeader* hdr, int num_sms,
+                     cudaStream_t stream) {
     using Cf = Cfg<WARPS>;
     auto kern = out_bf16 ? latent_attn_kernel<WARPS, true> : latent_attn_kernel<WARPS, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cf::SMEM));
@@ -249,23 +252,23 @@ cudaError_t launch_w(const void* Q, const void* KV, const int* idx, int B, int n
     if (grid < 1) grid = 1;
     kern<<<static_cast<int>(grid), WARPS * 32, Cf::SMEM, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(KV), idx, B, n_q, n_kv, Hq, topk,
-        scale * 1.4426950408889634f, O, hdr);
+        scale * 1.4426950408889634f, O, share, hdr);
     return cudaGetLastError();
 }
 
 }  // namespace lat
 
 cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
-                                      int Hq, int topk, float scale, void* O, bool out_bf16, WsHeader* hdr,
-                                      int num_sms, cudaStream_t stream) {
+                                      int Hq, int topk, float scale, void* O, bool out_bf16, IdxShare share,
+                                      WsHeader* hdr, int num_sms, cudaStream_t stream) {
     if (Hq % 64 == 0)
-        return lat::launch_w<8>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+        return lat::launch_w<8>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
     if (Hq % 32 == 0)
-        return lat::launch_w<4>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+        return lat::launch_w<4>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
     if (Hq % 16 == 0)
-        return lat::launch_w<2>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+        return lat::launch_w<2>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
     if (Hq % 8 == 0)
-        return lat::launch_w<1>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, hdr, num_sms, stream);
+        return lat::launch_w<1>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }
 

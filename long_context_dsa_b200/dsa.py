@@ -26,7 +26,7 @@ ABI_SYMBOLS = (
     "idx_score_topk_workspace_size", "idx_score_topk", "idx_scores",
     "idx_topk_scores_workspace_size", "idx_topk_scores",
     "idx_cache_init", "idx_cache_put", "idx_cache_get",
-    "sparse_attn_topk_workspace_size", "sparse_attn_topk",
+    "sparse_attn_topk_workspace_size", "sparse_attn_topk", "sparse_attn_topk_shared",
     "layer_group_forward_workspace_size", "layer_group_forward",
     "idx_score_topk_noalloc",
 )
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
         "idx_cache_get": ([ctypes.POINTER(IndexCacheStruct), i, ctypes.c_char_p, ctypes.POINTER(vp)], i),
         "sparse_attn_topk_workspace_size": ([i, i, i, i, i, i, i, i, psz], i),
         "sparse_attn_topk": ([vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, i, vp, sz, vp], i),
+        "sparse_attn_topk_shared": ([vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, f, vp, i, vp, sz, vp], i),
         "layer_group_forward_workspace_size": ([ctypes.POINTER(GroupShape), psz], i),
         "layer_group_forward": ([ctypes.POINTER(GroupShape), ctypes.POINTER(LayerArgs), i, ctypes.c_char_p,
                                  ctypes.POINTER(IndexCacheStruct), ctypes.POINTER(GroupStats), vp, sz, vp], i),
@@ -281,6 +282,37 @@ def sparse_attn_topk(Q, K, V, idx, scale: float | None = None, o_dtype=torch.flo
     _check(lib().sparse_attn_topk(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk,
                                   float(scale or 0.0), _ptr(out), od, _ptr(workspace), workspace.numel(),
                                   _stream(stream)))
+    return out
+
+
+def sparse_attn_topk_shared(Q, K, V, idx, q_per_idx: int, q_pos0: int, scale: float | None = None,
+                            o_dtype=torch.float32, d_v: int | None = None, out=None, workspace=None,
+                            stream=None) -> torch.Tensor:
+    """As sparse_attn_topk, but query row i uses index row idx[b, i // q_per_idx], causally limited to
+    its own position q_pos0 + i.  idx: [B, ceil(n_q / q_per_idx), topk]."""
+    _need(Q, torch.bfloat16, "Q")
+    _need(K, torch.bfloat16, "K")
+    if V is not None:
+        _need(V, torch.bfloat16, "V")
+    _need(idx, torch.int32, "idx")
+    B, n_q, Hq, d_qk = Q.shape
+    n_kv, Hkv = K.shape[1], K.shape[2]
+    if V is not None:
+        d_v = V.shape[3]
+    elif d_v is None:
+        raise ValueError("latent form (V=None) needs d_v")
+    if idx.shape[1] != (n_q + q_per_idx - 1) // q_per_idx:
+        raise ValueError("idx must have ceil(n_q / q_per_idx) rows per sequence")
+    topk = idx.shape[-1]
+    od = DSA_F32 if o_dtype == torch.float32 else DSA_BF16
+    if out is None:
+        out = torch.empty((B, n_q, Hq, d_v), dtype=o_dtype, device=Q.device)
+    _need(out, o_dtype, "out")
+    if workspace is None:
+        workspace = _workspace(sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk), Q.device)
+    _check(lib().sparse_attn_topk_shared(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), B, n_q, q_pos0, n_kv, Hq, Hkv, d_qk,
+                                         d_v, topk, q_per_idx, float(scale or 0.0), _ptr(out), od, _ptr(workspace),
+                                         workspace.numel(), _stream(stream)))
     return out
 
 

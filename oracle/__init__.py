@@ -19,6 +19,7 @@ from .dsa_oracle import (  # noqa: F401
     topk_select,
     IndexCache,
     sparse_attention,
+    sparse_attention_shared,
     layer_group_forward,
     topk_overlap,
     check_pattern,

@@ -259,6 +259,27 @@ def sparse_attention(Q, K, V, idx, scale: float | None = None, d_v: int | None =
 # a5: one layer group
 # ---------------------------------------------------------------------------
 
+def sparse_attention_shared(Q, K, V, idx_shared, q_per_idx: int, q_pos0: int, scale: float | None = None,
+                            d_v: int | None = None) -> np.ndarray:
+    """Several consecutive query tokens reuse one selection (multi-token decode).
+
+    [Term] §IndexShare: the same sharing that lets layers reuse one indexer
+    lifts MTP speculative-decoding acceptance.  Reading (the page gives no
+    more): query row i (absolute position q_pos0 + i) uses selection row
+    i // q_per_idx and, being causal, only the entries of that row at or
+    before its own position; then plain sparse attention.
+    idx_shared: int [ceil(n_q / q_per_idx), k].
+    """
+    idx_shared = np.asarray(idx_shared)
+    n_q = len(Q)
+    rows = []
+    for i in range(n_q):
+        r = idx_shared[i // q_per_idx].astype(np.int64).copy()
+        r[r > q_pos0 + i] = -1
+        rows.append(r)
+    return sparse_attention(Q, K, V, np.stack(rows), scale=scale, d_v=d_v)
+
+
 def layer_group_forward(layers, pattern: str, topk: int, q_pos0: int = 0,
                         scale: float | None = None):
     """Run a layer group: F layers index, S layers reuse, all layers attend.

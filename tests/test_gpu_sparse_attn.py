@@ -154,3 +154,52 @@ def test_latent_attention_matches_oracle(case):
     for b in range(B):
         ref = oracle.sparse_attention(Q[b, rows], KV[b], None, idx[b, rows], d_v=512)
         check_attention(O[b, rows], ref)
+
+
+# several query tokens per sequence reuse one selection (multi-token decode)
+# (name, B, n_q, q_pos0, n_kv, Hq, Hkv, d, k, q_per_idx)
+SHARED = [
+    ("mtp4_gqa", 3, 4, 2996, 3000, 32, 4, 128, 2048, 4),
+    ("mtp_ragged_d64", 2, 5, 995, 1000, 16, 2, 64, 300, 2),
+    ("mtp_b64_split_ranges", 64, 4, 1996, 2000, 32, 4, 128, 512, 4),
+    ("mtp_latent", 2, 3, 497, 500, 16, 1, 576, 128, 3),
+]
+
+
+def _shared_rows(B, n_q, q_pos0, n_kv, k, q, seed):
+    """Each group's selection is made for its last query (top-k of random scores up to that position)."""
+    rng = np.random.default_rng(seed)
+    n_rows = (n_q + q - 1) // q
+    out = np.empty((B, n_rows, k), np.int32)
+    for b in range(B):
+        for r in range(n_rows):
+            last = q_pos0 + min((r + 1) * q, n_q) - 1
+            sc = rng.standard_normal((1, n_kv)).astype(np.float32)
+            out[b, r] = oracle.topk_select(sc, k, last)[0]
+    return out
+
+
+@pytest.mark.parametrize("case", SHARED, ids=[c[0] for c in SHARED])
+def test_shared_selection_matches_oracle(case):
+    name, B, n_q, q_pos0, n_kv, Hq, Hkv, d, k, q = case
+    latent = d == 576
+    Q, K, V = synth.attention_inputs(name, 0, B, n_q, n_kv, Hq, Hkv, d, None if latent else d)
+    idx = _shared_rows(B, n_q, q_pos0, n_kv, k, q, 21)
+    d_v = 512 if latent else d
+    ws = torch.zeros(dsa.sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, Hkv, d, d_v, k), dtype=torch.uint8,
+                     device=DEV)
+    O = dsa.sparse_attn_topk_shared(Q.to(DEV), K.to(DEV), None if latent else V.to(DEV),
+                                    torch.from_numpy(idx).to(DEV), q, q_pos0, d_v=d_v, workspace=ws)
+    assert dsa.read_status(ws) == 0
+    O = O.cpu().numpy()
+    for b in range(B):
+        ref = oracle.sparse_attention_shared(Q[b], K[b], None if latent else V[b], idx[b], q, q_pos0,
+                                             d_v=d_v if latent else None)
+        check_attention(O[b], ref)
+
+
+def test_shared_rejects_positions_outside_the_cache():
+    Q, K, V = synth.attention_inputs("mtp_bad", 0, 1, 4, 100, 8, 8, 64, 64)
+    idx = np.zeros((1, 1, 8), np.int32)
+    with pytest.raises(dsa.DsaError):
+        dsa.sparse_attn_topk_shared(Q.to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV), 4, 97)

@@ -16,7 +16,7 @@ import torch
 
 import oracle
 from oracle import (IndexCache, check_pattern, e4m3_decode, indexer_scores,
-                    indexer_scores_fp8, layer_group_forward, sparse_attention,
+                    indexer_scores_fp8, layer_group_forward, sparse_attention, sparse_attention_shared,
                     topk_overlap, topk_select)
 from long_context_dsa_b200 import synth
 
@@ -325,6 +325,52 @@ def test_attention_invariant_to_order_and_padding_of_indices():
         pos = rng.choice(7, v.size, replace=False)
         shuffled[t, np.sort(pos)] = v
     assert np.allclose(sparse_attention(Q, K, V, idx), sparse_attention(Q, K, V, shuffled), atol=1e-14)
+
+
+def test_shared_selection_with_one_query_per_row_is_plain_attention():
+    rng = np.random.default_rng(16)
+    n, p0 = 10, 20
+    Q = rng.standard_normal((n, 4, 8))
+    K = rng.standard_normal((p0 + n, 2, 8))
+    V = rng.standard_normal((p0 + n, 2, 8))
+    idx = topk_select(rng.standard_normal((n, p0 + n)).astype(np.float32), 6, p0)
+    assert np.array_equal(sparse_attention_shared(Q, K, V, idx, 1, p0), sparse_attention(Q, K, V, idx))
+
+
+def test_shared_selection_of_every_token_is_dense_causal_attention():
+    """One shared row listing the whole prefix: each query of the group attends densely and
+    causally up to its own position (torch SDPA with an explicit mask, fp64)."""
+    rng = np.random.default_rng(17)
+    n, p0, Hq, Hkv, d = 5, 11, 4, 2, 8
+    Q = rng.standard_normal((n, Hq, d))
+    K = rng.standard_normal((p0 + n, Hkv, d))
+    V = rng.standard_normal((p0 + n, Hkv, d))
+    row = np.arange(p0 + n)[None, :]
+    got = sparse_attention_shared(Q, K, V, row, n, p0)
+    G = Hq // Hkv
+    mask = torch.from_numpy(np.arange(p0 + n)[None, :] <= (p0 + np.arange(n))[:, None])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q).permute(1, 0, 2), torch.from_numpy(K).repeat_interleave(G, 1).permute(1, 0, 2),
+        torch.from_numpy(V).repeat_interleave(G, 1).permute(1, 0, 2), attn_mask=mask).permute(1, 0, 2).numpy()
+    assert np.allclose(got, ref, atol=1e-12)
+
+
+def test_shared_selection_drops_entries_after_each_querys_position():
+    rng = np.random.default_rng(18)
+    n, p0 = 3, 6
+    Q = rng.standard_normal((n, 2, 4))
+    K = rng.standard_normal((p0 + n, 1, 4))
+    V = rng.standard_normal((p0 + n, 1, 4))
+    row = np.array([[1, 4, p0 + 1, p0 + 2, -1]])     # made for the group's last query
+    got = sparse_attention_shared(Q, K, V, row, n, p0)
+    assert np.array_equal(got[0], sparse_attention(Q[:1], K, V, np.array([[1, 4]]))[0])
+    assert np.array_equal(got[1], sparse_attention(Q[1:2], K, V, np.array([[1, 4, p0 + 1]]))[0])
+    assert np.array_equal(got[2], sparse_attention(Q[2:], K, V, np.array([[1, 4, p0 + 1, p0 + 2]]))[0])
+    # ragged groups: q_per_idx = 2 over 3 queries uses rows 0, 0, 1
+    rows2 = np.array([[0, 2, -1], [3, 5, p0 + 2]])
+    got2 = sparse_attention_shared(Q, K, V, rows2, 2, p0)
+    assert np.array_equal(got2[1], sparse_attention(Q[1:2], K, V, rows2[:1])[0])
+    assert np.array_equal(got2[2], sparse_attention(Q[2:], K, V, rows2[1:])[0])
 
 
 # --------------------------------------------------------------------------
