@@ -221,6 +221,36 @@ DSA_API int sparse_attn_topk_shared(const void* Q, const void* K, const void* V,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* ======================================================================
+ * F/S pattern search -- which layers of a group keep their indexer.
+ *
+ * [QbitAI] §IndexCache: for an existing model, the layers worth keeping are
+ * searched by the change in loss; [Explainer] §训练无关: a greedy pass over a
+ * small calibration batch picks the F and S layers, weights untouched.  The
+ * loss proxy here is selection overlap (the pages report 70-100% between
+ * adjacent layers): an S layer reusing F layer f's top-k loses the part of
+ * its own top-k that f's misses.  Steps: run every layer as F on calibration
+ * rows (idx_score_topk), measure overlaps (idx_overlap), search
+ * (layer_pattern_search), then run groups with the pattern found.
+ * ====================================================================== */
+
+/* counts[r] = |A_r ∩ B_r| for rows r of two [rows, topk] int32 index buffers
+ * in the canonical layout (ascending indices, then -1; as idx_score_topk
+ * writes them).  Device pointers; asynchronous on `stream`.  Rows out of the
+ * canonical layout give unspecified counts (never out-of-bounds reads). */
+DSA_API int idx_overlap(const int32_t* idx_a, const int32_t* idx_b, int64_t rows, int topk,
+                        int32_t* counts, void* stream);
+
+/* Greedy removal from the all-F pattern.  overlap: host [n_layers][n_layers]
+ * doubles, row-major, overlap[f][j] (f < j, in [0,1]) = mean fraction of
+ * layer j's selection that layer f's selection also holds; other entries are
+ * not read.  Loss of a pattern = sum over its S layers j of
+ * (1 - overlap[f][j]), f the most recent F layer before j.  While more than
+ * n_f layers are F, the F layer (never layer 0) whose turning into S gives the
+ * smallest loss becomes S (the lowest such layer on ties).  Writes n_layers
+ * characters 'F'/'S' and a terminating NUL to host pattern_out. */
+DSA_API int layer_pattern_search(const double* overlap, int n_layers, int n_f, char* pattern_out);
+
+/* ======================================================================
  * layer_group_forward -- one layer group: F layers index, S layers reuse.
  *
  * [QbitAI] §IndexCache: few layers keep an indexer, compute the top-k and

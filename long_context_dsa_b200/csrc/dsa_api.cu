@@ -23,6 +23,9 @@ cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* 
                                       WsHeader* hdr, int num_sms, cudaStream_t stream);
 size_t indexer_workspace_bytes(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype,
                                int num_sms);
+cudaError_t launch_overlap_count(const int* a, const int* b, long long rows, int k, int* out, int num_sms,
+                                 cudaStream_t stream);
+void greedy_pattern(const double* ov, int n, int n_f, char* out);
 size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms);
 cudaError_t launch_indexer(const void* q, const float* q_scale, const void* k, const float* k_scale,
                            const float* w, int dtype, int B, int n_q, int q_pos0, int n_kv, int H, int d,
@@ -266,6 +269,33 @@ int idx_cache_get(const dsa_index_cache* cache, int layer, const char* pattern, 
         return fail(DSA_ERR_INVALID_ARG, "layer %d needs indices from F layer %d, which has not written the cache",
                     layer, last_f);
     *idx = cache->buf;
+    return DSA_OK;
+}
+
+// ------------------------------------------------------------ F/S pattern search
+int idx_overlap(const int32_t* idx_a, const int32_t* idx_b, int64_t rows, int topk, int32_t* counts,
+                void* stream) {
+    if (!idx_a || !idx_b || !counts) return fail(DSA_ERR_INVALID_ARG, "NULL pointer");
+    if (rows < 1 || topk < 1) return fail(DSA_ERR_INVALID_ARG, "bad sizes rows=%lld topk=%d",
+                                          static_cast<long long>(rows), topk);
+    int sms;
+    int rc = sm_count(&sms);
+    if (rc) return rc;
+    cudaError_t e = launch_overlap_count(idx_a, idx_b, rows, topk, counts, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "idx_overlap");
+    return DSA_OK;
+}
+
+int layer_pattern_search(const double* overlap, int n_layers, int n_f, char* pattern_out) {
+    if (!overlap || !pattern_out) return fail(DSA_ERR_INVALID_ARG, "NULL pointer");
+    if (n_layers < 1 || n_layers > 4096) return fail(DSA_ERR_INVALID_ARG, "n_layers %d out of range", n_layers);
+    if (n_f < 1 || n_f > n_layers) return fail(DSA_ERR_INVALID_ARG, "n_f %d not in [1, %d]", n_f, n_layers);
+    for (int f = 0; f < n_layers; ++f)
+        for (int j = f + 1; j < n_layers; ++j) {
+            const double v = overlap[static_cast<size_t>(f) * n_layers + j];
+            if (!(v >= 0.0 && v <= 1.0)) return fail(DSA_ERR_INVALID_ARG, "overlap[%d][%d] not in [0, 1]", f, j);
+        }
+    greedy_pattern(overlap, n_layers, n_f, pattern_out);
     return DSA_OK;
 }
 

@@ -28,7 +28,7 @@ ABI_SYMBOLS = (
     "idx_cache_init", "idx_cache_put", "idx_cache_get",
     "sparse_attn_topk_workspace_size", "sparse_attn_topk", "sparse_attn_topk_shared",
     "layer_group_forward_workspace_size", "layer_group_forward",
-    "idx_score_topk_noalloc",
+    "idx_score_topk_noalloc", "idx_overlap", "layer_pattern_search",
 )
 
 
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         "layer_group_forward": ([ctypes.POINTER(GroupShape), ctypes.POINTER(LayerArgs), i, ctypes.c_char_p,
                                  ctypes.POINTER(IndexCacheStruct), ctypes.POINTER(GroupStats), vp, sz, vp], i),
         "idx_score_topk_noalloc": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp], i),
+        "idx_overlap": ([vp, vp, i64, i, vp, vp], i),
+        "layer_pattern_search": ([ctypes.POINTER(ctypes.c_double), i, i, ctypes.c_char_p], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -314,6 +316,34 @@ def sparse_attn_topk_shared(Q, K, V, idx, q_per_idx: int, q_pos0: int, scale: fl
                                          d_v, topk, q_per_idx, float(scale or 0.0), _ptr(out), od, _ptr(workspace),
                                          workspace.numel(), _stream(stream)))
     return out
+
+
+# -------------------------------------------------------------- F/S pattern search
+def idx_overlap(idx_a: torch.Tensor, idx_b: torch.Tensor, counts=None, stream=None) -> torch.Tensor:
+    """Per-row |A ∩ B| of two canonical index buffers [..., topk] (int32 counts, one per row)."""
+    _need(idx_a, torch.int32, "idx_a")
+    _need(idx_b, torch.int32, "idx_b")
+    if idx_a.shape != idx_b.shape:
+        raise ValueError("index buffers differ in shape")
+    topk = idx_a.shape[-1]
+    rows = idx_a.numel() // topk
+    if counts is None:
+        counts = torch.empty(rows, dtype=torch.int32, device=idx_a.device)
+    _check(lib().idx_overlap(_ptr(idx_a), _ptr(idx_b), rows, topk, _ptr(counts), _stream(stream)))
+    return counts
+
+
+def layer_pattern_search(overlap, n_f: int) -> str:
+    """Greedy F/S pattern with n_f F layers from a host [n_layers, n_layers] overlap matrix."""
+    import numpy as np
+
+    ov = np.ascontiguousarray(np.asarray(overlap, dtype=np.float64))
+    n = ov.shape[0]
+    if ov.shape != (n, n):
+        raise ValueError("overlap must be square")
+    buf = ctypes.create_string_buffer(n + 1)
+    _check(lib().layer_pattern_search(ov.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), n, n_f, buf))
+    return buf.value.decode()
 
 
 # -------------------------------------------------------------- layer group

@@ -102,6 +102,29 @@ class StructuredIndexer:
         return q.to(torch.bfloat16), self.w[:, t0:t1].contiguous()
 
 
+class SegmentedIndexer:
+    """Indexer inputs of a layer group whose layers fall into segments: the layers of one
+    segment share one StructuredIndexer's token structure and head weights (their top-k
+    selections overlap strongly), while each segment draws its own (selections of layers in
+    different segments barely overlap).  A stand-in for a model whose layers change what they
+    attend to at a few depths, the case a search over F/S patterns has to find.
+    ``segment_starts`` lists the first layer of each segment and starts with 0."""
+
+    def __init__(self, name: str, B: int, L: int, H: int, d: int, r: int, base_std: float, noise_std: float,
+                 segment_starts, device="cpu", seed: int = 0):
+        starts = list(segment_starts)
+        assert starts and starts[0] == 0 and starts == sorted(set(starts))
+        self.starts = starts
+        self.parts = [StructuredIndexer(f"{name}/segment{i}", B, L, H, d, r, base_std, noise_std, device, seed)
+                      for i in range(len(starts))]
+
+    def segment(self, l: int) -> int:
+        return max(i for i, s in enumerate(self.starts) if s <= l)
+
+    def layer(self, l: int):
+        return self.parts[self.segment(l)].layer(l)
+
+
 def attention_inputs(name: str, l: int, B: int, L_q: int, L_kv: int, Hq: int, Hkv: int,
                      d_qk: int, d_v: int | None, device="cpu", seed: int = 0):
     """Q [B, L_q, Hq, d_qk], K [B, L_kv, Hkv, d_qk], V [B, L_kv, Hkv, d_v] (None if d_v is None), bf16."""

@@ -23,4 +23,7 @@ from .dsa_oracle import (  # noqa: F401
     layer_group_forward,
     topk_overlap,
     check_pattern,
+    overlap_counts,
+    pattern_loss,
+    pattern_search,
 )

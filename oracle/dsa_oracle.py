@@ -331,3 +331,55 @@ def topk_overlap(idx_a, idx_b, k: int, q_pos0: int = 0) -> float:
             continue
         fr.append(np.intersect1d(a[i][a[i] >= 0], b[i][b[i] >= 0]).size / k)
     return float(np.mean(fr)) if fr else 1.0
+
+
+# ---------------------------------------------------------------------------
+# F/S pattern search (which layers keep their indexer)
+# ---------------------------------------------------------------------------
+
+def overlap_counts(idx_a, idx_b) -> np.ndarray:
+    """Per row, the number of token indices (entries >= 0) both selections hold."""
+    a = np.asarray(idx_a)
+    b = np.asarray(idx_b)
+    out = np.zeros(a.shape[0], dtype=np.int64)
+    for i in range(a.shape[0]):
+        sa = {int(x) for x in a[i] if x >= 0}
+        out[i] = sum(1 for x in b[i] if x >= 0 and int(x) in sa)
+    return out
+
+
+def pattern_loss(overlap, pattern: str) -> float:
+    """Proxy loss of a pattern: each S layer j loses 1 - overlap[f][j] of its own selection,
+    f being the most recent F layer before it (the layer whose indices it reuses)."""
+    check_pattern(pattern)
+    total, f = 0.0, 0
+    for j, c in enumerate(pattern):
+        if c == "F":
+            f = j
+        else:
+            total += 1.0 - float(overlap[f][j])
+    return total
+
+
+def pattern_search(overlap, n_f: int) -> str:
+    """Greedy F/S choice ([QbitAI] §IndexCache: search which layers to keep by the change in
+    loss; [Explainer] §训练无关: a greedy algorithm over calibration data picks the layers).
+
+    Reading: start with every layer F; while more than n_f are F, make S the F layer (not
+    layer 0, which must index) whose change raises pattern_loss least, the lowest layer on ties.
+    """
+    n = len(overlap)
+    assert 1 <= n_f <= n
+    pat = ["F"] * n
+    while pat.count("F") > n_f:
+        best, best_loss = None, None
+        for l in range(1, n):
+            if pat[l] != "F":
+                continue
+            trial = pat.copy()
+            trial[l] = "S"
+            loss = pattern_loss(overlap, "".join(trial))
+            if best is None or loss < best_loss:
+                best, best_loss = l, loss
+        pat[best] = "S"
+    return "".join(pat)

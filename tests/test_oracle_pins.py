@@ -377,6 +377,39 @@ def test_shared_selection_drops_entries_after_each_querys_position():
 # pattern, cache, layer group, chunking, overlap
 # --------------------------------------------------------------------------
 
+def test_overlap_counts_fixture():
+    a = np.array([[0, 3, 5, 9, -1], [1, 2, 3, 4, 5], [-1, -1, -1, -1, -1]])
+    b = np.array([[3, 4, 9, -1, -1], [0, 6, 7, 8, 9], [-1, -1, -1, -1, -1]])
+    assert list(oracle.overlap_counts(a, b)) == [2, 0, 0]
+
+
+def test_pattern_search_hand_worked_four_layers():
+    """All-F loss 0.  One removal: layer 1 costs 0.1, layer 2 costs 1-0.6 = 0.4 (it reuses layer 1),
+    layer 3 costs 0.05 -> FFFS.  Second removal: layer 1 gives 0.1 + 0.05 = 0.15, layer 2 gives
+    (1-0.6) + (1-0.5) = 0.9 -> FSFS.  Third: FSSS."""
+    ov = np.zeros((4, 4))
+    ov[0, 1], ov[0, 2], ov[1, 2], ov[0, 3], ov[1, 3], ov[2, 3] = 0.9, 0.5, 0.6, 0.4, 0.5, 0.95
+    assert oracle.pattern_search(ov, 4) == "FFFF"
+    assert oracle.pattern_search(ov, 3) == "FFFS"
+    assert oracle.pattern_search(ov, 2) == "FSFS"
+    assert oracle.pattern_search(ov, 1) == "FSSS"
+    assert oracle.pattern_loss(ov, "FSFS") == pytest.approx(0.15)
+
+
+def test_pattern_search_finds_segment_starts_and_the_optimum():
+    """Layers in blocks (0.9 inside a block, 0.3 across): with one F per block the greedy
+    keeps exactly the block starts, which brute force over all patterns confirms is optimal."""
+    import itertools
+    blocks = [0, 0, 0, 1, 1, 1, 2, 2]
+    n = len(blocks)
+    ov = np.array([[0.9 if blocks[i] == blocks[j] else 0.3 for j in range(n)] for i in range(n)])
+    got = oracle.pattern_search(ov, 3)
+    assert got == "FSSFSSFS"
+    best = min(("F" + "".join("F" if i + 1 in c else "S" for i in range(n - 1))
+                for c in itertools.combinations(range(1, n), 2)), key=lambda p: oracle.pattern_loss(ov, p))
+    assert oracle.pattern_loss(ov, got) == pytest.approx(oracle.pattern_loss(ov, best))
+
+
 @pytest.mark.parametrize("bad", ["", "S", "SFFF", "FXS", "fsss"])
 def test_pattern_rejects(bad):
     with pytest.raises(ValueError):
