@@ -550,6 +550,98 @@ def run_mtp(args, dev):
             "speedup": round(res["unshared"] / res["shared"], 3)}
 
 
+def run_paged(args, dev):
+    """Serving-style decode: 64 sequences of different lengths (seeded, 100K-200K tokens) whose
+    k_I and K/V caches sit in a shared pool of 64-token pages in shuffled order; one new token each,
+    4 layers FSSS (paged decode indexer once, paged gather attention on every layer)."""
+    import numpy as np
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    B, Lmax, P, nl = 64, 200000, 64, 4
+    rng = np.random.default_rng(4000)
+    lens = rng.integers(100000, Lmax + 1, size=B).astype(np.int32)
+    pages = (lens + P - 1) // P
+    num_pages = int(pages.sum())
+    max_pages = int(pages.max())
+    perm = torch.from_numpy(rng.permutation(num_pages).astype(np.int64)).to(dev)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    rows = []  # pool row of every cached token, sequence by sequence
+    off = 0
+    for b in range(B):
+        table[b, :pages[b]] = torch.arange(off, off + pages[b], dtype=torch.int32)
+        off += int(pages[b])
+    table = table.to(dev)
+    table = torch.where(table >= 0, perm[table.clamp(min=0).long()].int(), table)
+    for b in range(B):
+        t = torch.arange(int(lens[b]), device=dev)
+        rows.append(table[b, t // P].long() * P + t % P)
+
+    def to_pool(x):  # [B, Lmax, ...] contiguous cache -> [num_pages * P, ...] pool
+        pool = torch.zeros((num_pages * P,) + tuple(x.shape[2:]), dtype=x.dtype, device=dev)
+        for b in range(B):
+            pool[rows[b]] = x[b, :int(lens[b])]
+        return pool
+
+    gen = synth.StructuredIndexer("paged200k", B, Lmax, H_I, D_I, r=32, base_std=1.0, noise_std=0.2, device=dev,
+                                  seed=4000)
+    k_pool = to_pool(gen.keys(0)).view(num_pages, P, D_I)
+    q = torch.stack([gen.queries(0, int(n) - 1, int(n))[0][b, 0] for b, n in enumerate(lens)]).contiguous()
+    w = torch.stack([gen.w[b, int(n) - 1] for b, n in enumerate(lens)]).contiguous()
+    del gen
+    layers = []
+    for l in range(nl):
+        _, K, V = synth.attention_inputs("paged200k", l, B, 1, Lmax, HQ, HKV, DH, DH, device=dev, seed=4000)
+        Kp = to_pool(K).view(num_pages, P, HKV, DH)
+        del K
+        Vp = to_pool(V).view(num_pages, P, HKV, DH)
+        del V
+        Q = synth.normal((B, HQ, DH), synth.seed_for(4000, "paged200k", l, "Qdec"), dev, dtype=torch.bfloat16)
+        layers.append((Q, Kp, Vp))
+        torch.cuda.empty_cache()
+    seq = torch.from_numpy(lens).to(dev)
+    idx = torch.empty((B, TOPK), dtype=torch.int32, device=dev)
+    O = torch.empty((B, HQ, DH), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(max(dsa.idx_score_topk_paged_workspace_size(B, Lmax, H_I, D_I, TOPK),
+                         dsa.sparse_attn_topk_workspace_size(B, 1, num_pages * P, HQ, HKV, DH, DH, TOPK)),
+                     dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record()
+        dsa.idx_score_topk_paged(q, k_pool, table, seq, w, TOPK, Lmax, out=idx, workspace=ws)
+        if evs:
+            evs[1].record()
+        for (Q, Kp, Vp) in layers:
+            dsa.sparse_attn_topk_paged(Q, Kp, Vp, table, seq, idx, o_dtype=torch.bfloat16, out=O, workspace=ws)
+        if evs:
+            evs[2].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = 10
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(n):
+        step(evs if i == n - 1 else None)
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b) / n
+    kbytes = int(lens.sum()) * D_I * 2
+    del layers, k_pool
+    torch.cuda.empty_cache()
+    return {"workload": f"paged decode: B={B} sequences of {int(lens.min())}-{int(lens.max())} tokens "
+                        f"(mean {int(lens.mean())}) in shuffled {P}-token pages, 4 layers FSSS, "
+                        f"H_I={H_I} d_I={D_I} top-{TOPK}, GQA {HQ}Q/{HKV}KV d={DH}",
+            "tok_per_s": round(B / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "indexer_ms": round(evs[0].elapsed_time(evs[1]), 4),
+            "attention_ms": round(evs[1].elapsed_time(evs[2]), 4),
+            "indexer_gbs": round(kbytes / (evs[0].elapsed_time(evs[1]) / 1e3) / 1e9, 1)}
+
+
 def run_ctx1m(args, dev):
     """The last 8192-token chunk of a 1M-token chunked prefill: fp8 indexer (H_I=64, d_I=128,
     per-token scales) on 2 of 8 layers (FSSSFSSS), latent attention (576-dim rows, 512-dim values,
@@ -619,17 +711,17 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
-    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "ctx1m", "mtp"],
+    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "ctx1m", "mtp", "paged"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m: only that "
                          "extra measurement, printed as one JSON line")
     args = ap.parse_args()
     if args.case == "profile":
         run_profile_case(args)
         return
-    if args.case in ("decode", "ctx1m", "mtp"):
+    if args.case in ("decode", "ctx1m", "mtp", "paged"):
         import torch
         dev = torch.device("cuda", 0)
-        fn = {"decode": run_decode, "ctx1m": run_ctx1m, "mtp": run_mtp}[args.case]
+        fn = {"decode": run_decode, "ctx1m": run_ctx1m, "mtp": run_mtp, "paged": run_paged}[args.case]
         print(json.dumps({"case": args.case, **fn(args, dev)}), flush=True)
         return
 
@@ -662,6 +754,7 @@ def main():
         dev = torch.device("cuda", local_rank)
         out["decode"] = run_decode(args, dev)
         out["multi_token_decode"] = run_mtp(args, dev)
+        out["paged_decode"] = run_paged(args, dev)
         out["context_1m_tail_chunk"] = run_ctx1m(args, dev)
     if world > 1:
         import torch.distributed as dist

@@ -221,6 +221,48 @@ DSA_API int sparse_attn_topk_shared(const void* Q, const void* K, const void* V,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* ======================================================================
+ * Paged, variable-length decode (serving).
+ *
+ * The same decode-step operations ([QbitAI] §IndexCache: the indexer picks
+ * each new token's important history tokens; [Explainer] §稀疏注意力: the
+ * attention reads only those) over a batch of sequences of different
+ * lengths whose caches live in a shared pool of fixed-size pages.  Token t
+ * of sequence b is row page_table[b * max_pages + t / page_size] *
+ * page_size + t % page_size of the pool; seq_lens[b] counts its cached
+ * tokens, the new token (the query) being the last of them.
+ *
+ * idx_score_topk_paged: one query per sequence.
+ *   q_I        [B, H_I, d_I] bf16        w [B, H_I] fp32
+ *   k_pages    [num_pages * page_size, d_I] bf16
+ *   page_table [B, max_pages] int32 (device), seq_lens [B] int32 (device)
+ *   idx_out    [B, topk] int32: logical token indices, ascending, then -1.
+ * Requires H_I in {32, 64}, d_I = 128, page_size a power of two >= 16,
+ * max_pages * page_size >= max_seq_len >= every seq_lens[b] >= 1 (a length
+ * outside [1, max_pages * page_size] is flagged DSA_STATUS_BAD_INDEX and
+ * clamped; page numbers outside [0, num_pages) read page 0, whose keys are
+ * masked).  max_seq_len (host) sizes the work split.
+ *
+ * sparse_attn_topk_paged: attention of each sequence's query over its
+ * selected tokens (logical indices, as idx_score_topk_paged writes them).
+ *   Q [B, Hq, d] bf16; K_pages, V_pages [num_pages * page_size, Hkv, d]
+ *   bf16; idx [B, topk]; O [B, Hq, d] fp32 or bf16.  d in {64, 128},
+ *   Hq/Hkv <= 8.  Indices >= seq_lens[b] or mapping to a page outside
+ *   [0, num_pages) are skipped and flagged.  Workspace:
+ *   sparse_attn_topk_workspace_size(B, 1, num_pages * page_size, ...).
+ * ====================================================================== */
+DSA_API int idx_score_topk_paged_workspace_size(int B, int max_seq_len, int H_I, int d_I, int topk,
+                                                size_t* bytes);
+DSA_API int idx_score_topk_paged(const void* q_I, const void* k_pages, const int32_t* page_table,
+                                 const int32_t* seq_lens, const float* w, int B, int max_seq_len,
+                                 int page_size, int num_pages, int max_pages, int H_I, int d_I, int topk,
+                                 int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
+DSA_API int sparse_attn_topk_paged(const void* Q, const void* K_pages, const void* V_pages,
+                                   const int32_t* page_table, const int32_t* seq_lens, const int32_t* idx,
+                                   int B, int page_size, int num_pages, int max_pages, int Hq, int Hkv,
+                                   int d, int topk, float scale, void* O, int o_dtype,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ======================================================================
  * F/S pattern search -- which layers of a group keep their indexer.
  *
  * [QbitAI] §IndexCache: for an existing model, the layers worth keeping are

@@ -17,7 +17,12 @@ cudaError_t launch_topk_scores(const float* scores, int rows, int q_pos0, int n_
                                WsHeader* hdr, int num_sms, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, const int* idx, int B, int n_q,
                                int n_kv, int Hq, int Hkv, int d, int topk, float scale, void* O, bool out_bf16,
-                               IdxShare share, WsHeader* hdr, int num_sms, cudaStream_t stream);
+                               IdxShare share, KvPages pg, WsHeader* hdr, int num_sms, cudaStream_t stream);
+cudaError_t launch_indexer_decode_paged(const void* q, const void* k_pages, const int* page_table, const int* seq_lens,
+                                        const float* w, int B, int max_len, int page_size, int num_pages,
+                                        int max_pages, int H, int topk, int* idx_out, void* ws, int num_sms,
+                                        cudaStream_t stream);
+size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms);
 cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
                                       int Hq, int topk, float scale, void* O, bool out_bf16, IdxShare share,
                                       WsHeader* hdr, int num_sms, cudaStream_t stream);
@@ -319,7 +324,7 @@ int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, i
 namespace {
 int attn_common(const void* Q, const void* K, const void* V, const int32_t* idx, int B, int n_q, int n_kv, int Hq,
                 int Hkv, int d_qk, int d_v, int topk, float scale, void* O, int o_dtype, dsa::IdxShare share,
-                void* workspace, size_t workspace_bytes, void* stream) {
+                void* workspace, size_t workspace_bytes, void* stream, dsa::KvPages pages = dsa::kContiguous) {
     int rc = check_attn_shape(V, B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk);
     if (rc) return rc;
     if (!Q || !K || !idx || !O) return fail(DSA_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -333,12 +338,14 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* idx,
     int sms;
     if ((rc = sm_count(&sms))) return rc;
     cudaError_t e;
+    if (V == nullptr && pages.table) return fail(DSA_ERR_UNSUPPORTED, "paged caches need the separate K/V form");
     if (V == nullptr)
         e = launch_sparse_attn_latent(Q, K, idx, B, n_q, n_kv, Hq, topk, scale, O, o_dtype == DSA_BF16, share,
                                       static_cast<WsHeader*>(workspace), sms, static_cast<cudaStream_t>(stream));
     else
         e = launch_sparse_attn(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, d_qk, topk, scale, O, o_dtype == DSA_BF16,
-                               share, static_cast<WsHeader*>(workspace), sms, static_cast<cudaStream_t>(stream));
+                               share, pages, static_cast<WsHeader*>(workspace), sms,
+                               static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "sparse_attn_topk");
     return DSA_OK;
 }
@@ -349,6 +356,58 @@ int sparse_attn_topk(const void* Q, const void* K, const void* V, const int32_t*
                      void* workspace, size_t workspace_bytes, void* stream) {
     return attn_common(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, d_qk, d_v, topk, scale, O, o_dtype, dsa::kNoShare,
                        workspace, workspace_bytes, stream);
+}
+
+int sparse_attn_topk_paged(const void* Q, const void* K_pages, const void* V_pages, const int32_t* page_table,
+                           const int32_t* seq_lens, const int32_t* idx, int B, int page_size, int num_pages,
+                           int max_pages, int Hq, int Hkv, int d, int topk, float scale, void* O, int o_dtype,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (!page_table || !seq_lens || !V_pages) return fail(DSA_ERR_INVALID_ARG, "NULL page table, lengths or V");
+    if (page_size < 1 || num_pages < 1 || max_pages < 1)
+        return fail(DSA_ERR_INVALID_ARG, "bad page geometry page_size=%d num_pages=%d max_pages=%d", page_size,
+                    num_pages, max_pages);
+    const long long pool = static_cast<long long>(num_pages) * page_size;
+    if (pool > 0x7fffffffll) return fail(DSA_ERR_INVALID_ARG, "page pool too large");
+    const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages};
+    return attn_common(Q, K_pages, V_pages, idx, B, 1, static_cast<int>(pool), Hq, Hkv, d, d, topk, scale, O,
+                       o_dtype, dsa::kNoShare, workspace, workspace_bytes, stream, pages);
+}
+
+int idx_score_topk_paged_workspace_size(int B, int max_seq_len, int H_I, int d_I, int topk, size_t* bytes) {
+    if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
+    if (B < 1 || max_seq_len < 1 || topk < 1 || topk > DSA_TOPK_MAX)
+        return fail(DSA_ERR_INVALID_ARG, "bad sizes");
+    if (!((H_I == 32 || H_I == 64) && d_I == 128))
+        return fail(DSA_ERR_UNSUPPORTED, "paged decode indexer supports H_I in {32, 64}, d_I = 128");
+    int sms;
+    int rc = sm_count(&sms);
+    if (rc) return rc;
+    *bytes = kWsHeaderBytes + indexer_decode_workspace_bytes(B, max_seq_len - 1, topk, sms);
+    return DSA_OK;
+}
+
+int idx_score_topk_paged(const void* q_I, const void* k_pages, const int32_t* page_table, const int32_t* seq_lens,
+                         const float* w, int B, int max_seq_len, int page_size, int num_pages, int max_pages,
+                         int H_I, int d_I, int topk, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    if (!q_I || !k_pages || !page_table || !seq_lens || !w || !idx_out) return fail(DSA_ERR_INVALID_ARG, "NULL pointer");
+    if (page_size < 16 || (page_size & (page_size - 1)) != 0)
+        return fail(DSA_ERR_INVALID_ARG, "page_size %d must be a power of two >= 16", page_size);
+    if (num_pages < 1 || max_pages < 1 || static_cast<long long>(max_pages) * page_size < max_seq_len)
+        return fail(DSA_ERR_INVALID_ARG, "page table cannot hold max_seq_len tokens");
+    if (static_cast<long long>(num_pages) * page_size > 0x7fffffffll) return fail(DSA_ERR_INVALID_ARG, "page pool too large");
+    if (!aligned16(q_I) || !aligned16(k_pages)) return fail(DSA_ERR_INVALID_ARG, "q_I and k_pages must be 16-byte aligned");
+    size_t need;
+    int rc = idx_score_topk_paged_workspace_size(B, max_seq_len, H_I, d_I, topk, &need);
+    if (rc) return rc;
+    if ((rc = check_ws(workspace, workspace_bytes, need))) return rc;
+    int sms;
+    if ((rc = sm_count(&sms))) return rc;
+    cudaError_t e = launch_indexer_decode_paged(q_I, k_pages, page_table, seq_lens, w, B, max_seq_len, page_size,
+                                                num_pages, max_pages, H_I, topk, idx_out, workspace, sms,
+                                                static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "idx_score_topk_paged");
+    return DSA_OK;
 }
 
 int sparse_attn_topk_shared(const void* Q, const void* K, const void* V, const int32_t* idx, int B, int n_q,

@@ -41,6 +41,17 @@ struct IdxShare {
 };
 static constexpr IdxShare kNoShare = {1, 0, 0};
 
+// Paged K/V cache (serving): token t of sequence b lives in row
+// table[b * max_pages + t / page_size] * page_size + t % page_size of a
+// [num_pages * page_size, ...] pool; lens[b] is the sequence's cache length.
+// table == NULL: the contiguous [B, n_kv, ...] layout.
+struct KvPages {
+    const int* table;
+    const int* lens;
+    int page_size, max_pages, num_pages;
+};
+static constexpr KvPages kContiguous = {nullptr, nullptr, 0, 0, 0};
+
 // Nanoseconds from the global timer.
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;

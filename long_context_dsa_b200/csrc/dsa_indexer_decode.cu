@@ -16,6 +16,10 @@
 //   * Each unit writes its partial top-k (ascending indices with their score
 //     keys); topk_merge_pairs then selects the final top-k of each sequence
 //     from its units' lists (dsa_topk_scores.cu).
+//   * The key cache may be paged (serving: fixed-size pages of tokens, a page
+//     table per sequence) and sequences may differ in length: each 128-key
+//     tile is fetched page by page, keys past a sequence's length are masked,
+//     and units past a sequence's last tile select nothing.
 #include <cuda.h>
 
 #include "dsa_tc.cuh"
@@ -52,6 +56,9 @@ struct DecCfg {
 
 struct DecParams {
     const float* w;
+    const int* seq_lens;    // [B] cache length of each sequence, or NULL: every sequence has q_pos0 + 1 keys
+    const int* page_table;  // [B, max_pages] physical page of each logical page, or NULL: contiguous [B, n_kv]
+    int page_size, max_pages, num_pages;
     int B, q_pos0, n_kv, topk, splits, tiles_per_split;
     uint32_t* part_key;  // [B * splits, topk]
     int* part_idx;       // [B * splits, topk]
@@ -86,7 +93,6 @@ __global__ void __launch_bounds__(192, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int units = p.B * p.splits;
-    const int nkt = (p.q_pos0 + 1 + 127) / 128;  // key tiles of a sequence (keys 0..q_pos0)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -117,11 +123,23 @@ __global__ void __launch_bounds__(192, 1)
     tc::fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
 
-    auto unit_range = [&](int u, int& b, int& j0, int& j1) {
+    // keys of sequence b (its query sits at the last of them); out-of-range lengths are flagged and clamped
+    auto seq_len = [&](int b) -> int {
+        if (!p.seq_lens) return p.q_pos0 + 1;
+        int len = __ldg(p.seq_lens + b);
+        const int cap = p.page_table ? p.max_pages * p.page_size : p.n_kv;
+        if (len < 1 || len > cap) {
+            if (threadIdx.x == 0) raise_status(p.hdr, DSA_STATUS_BAD_INDEX, len);
+            len = len < 1 ? 1 : cap;
+        }
+        return len;
+    };
+    auto unit_range = [&](int u, int& b, int& j0, int& j1, int& len) {
         b = u / p.splits;
+        len = seq_len(b);
         const int sp = u % p.splits;
         j0 = sp * p.tiles_per_split;
-        j1 = min(nkt, j0 + p.tiles_per_split);
+        j1 = min((len + 127) / 128, j0 + p.tiles_per_split);  // empty when the sequence is shorter
     };
 
     if (warp == 4) {
@@ -131,8 +149,8 @@ __global__ void __launch_bounds__(192, 1)
             bool ok = true;
             int pend_q = -1;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++wt) {
-                int b, j0, j1;
-                unit_range(u, b, j0, j1);
+                int b, j0, j1, len;
+                unit_range(u, b, j0, j1, len);
                 if (wt > 0 && !mbar_wait(q_empty, (wt - 1) & 1)) { ok = false; break; }
                 mbar_arrive_expect_tx(q_full, C::B_BYTES);
                 for (int kb = 0; kb < 2; ++kb) tc::tma_load_2d(sB + kb * H * 128, &tmap_q, kb * 64, b * H, q_full);
@@ -142,9 +160,26 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t rr = it / C::STAGES;
                     if (rr > 0 && !mbar_wait(&kv_empty[s], (rr - 1) & 1)) { ok = false; break; }
                     mbar_arrive_expect_tx(&kv_full[s], C::A_STAGE);
-                    for (int kb = 0; kb < 2; ++kb)
-                        tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128, &tmap_k, kb * 64, b * p.n_kv + j * 128,
-                                        &kv_full[s]);
+                    if (!p.page_table) {
+                        for (int kb = 0; kb < 2; ++kb)
+                            tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128, &tmap_k, kb * 64,
+                                            b * p.n_kv + j * 128, &kv_full[s]);
+                    } else {
+                        // the tile's 128 keys page by page (rows = pieces of min(page, 128) keys; the
+                        // pieces start at 1024-byte multiples, so the 128-byte swizzle lines up)
+                        const int piece = min(p.page_size, 128);
+                        const int used = (len + p.page_size - 1) / p.page_size;  // pages the sequence holds
+                        for (int r0 = 0; r0 < 128; r0 += piece) {
+                            const int tok = j * 128 + r0;
+                            const int lp = tok / p.page_size;
+                            int pg = lp < used ? __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages + lp) : 0;
+                            if (pg < 0 || pg >= p.num_pages) pg = 0;  // keys there are masked anyway
+                            const int row = pg * p.page_size + tok % p.page_size;
+                            for (int kb = 0; kb < 2; ++kb)
+                                tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128 + r0 * 128, &tmap_k, kb * 64,
+                                                row, &kv_full[s]);
+                        }
+                    }
                     if (*reinterpret_cast<volatile int*>(abort_flag)) { ok = false; ++it; break; }
                 }
             }
@@ -163,8 +198,8 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t it = 0, wt = 0, ua = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++wt) {
-                int b, j0, j1;
-                unit_range(u, b, j0, j1);
+                int b, j0, j1, len;
+                unit_range(u, b, j0, j1, len);
                 (void)b;
                 if (!mbar_wait(q_full, wt & 1)) { ok = false; break; }
                 tc::fence_after_sync();
@@ -204,8 +239,8 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t ua = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            int b, j0, j1;
-            unit_range(u, b, j0, j1);
+            int b, j0, j1, len;
+            unit_range(u, b, j0, j1, len);
             if (tid < H) ws[tid] = p.w[static_cast<size_t>(b) * H + tid];
             if (tid == 0) topk_row_init(st);
             grp.sync();
@@ -244,7 +279,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int s_key = j * 128 + tid;
                 const uint32_t key = score_key(sc_v);
                 const uint32_t tk = st->thr_key;
-                const bool adm = got & (s_key <= p.q_pos0) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
+                const bool adm = got & (s_key < len) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
                 topk_append_warp(wkey, widx, cnt, key, s_key, adm, sub);
                 if (((j - j0) % CHECK) == CHECK - 1 || j == j1 - 1) {
                     if (lane == 0) st->cnt[warp] = cnt;
@@ -288,6 +323,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+    // [rows, 128] bf16, 128-byte swizzled boxes of 64 columns x box_rows
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
         void* ptr = nullptr;
@@ -314,17 +350,34 @@ int dec_splits(int B, int nkt, int num_sms) {
     return s;
 }
 
+// Cache geometry of a decode launch.  Contiguous: k [B, n_kv, d], every sequence q_pos0 + 1 keys.
+// Paged: k [num_pages * page_size, d], page_table [B, max_pages], seq_lens [B] (device), at most
+// max_len keys a sequence (host bound that sizes the split).
+struct DecCache {
+    const int* seq_lens;
+    const int* page_table;
+    int page_size, max_pages, num_pages, max_len;
+};
+
 template <int H>
 cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int topk,
-                         int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
+                         const DecCache& pc, int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
     using C = DecCfg<H>;
     CUtensorMap mq, mk;
+    const bool paged = pc.page_table != nullptr;
+    const uint64_t krows = paged ? static_cast<uint64_t>(pc.num_pages) * pc.page_size : static_cast<uint64_t>(B) * n_kv;
     if (!make_map_dec(&mq, q, static_cast<uint64_t>(B) * H, H) ||
-        !make_map_dec(&mk, k, static_cast<uint64_t>(B) * n_kv, 128))
+        !make_map_dec(&mk, k, krows, paged ? static_cast<uint32_t>(pc.page_size < 128 ? pc.page_size : 128) : 128))
         return cudaErrorInvalidValue;
-    const int nkt = (q_pos0 + 1 + 127) / 128;
+    const int max_len = pc.seq_lens ? pc.max_len : q_pos0 + 1;
+    const int nkt = (max_len + 127) / 128;
     DecParams p;
     p.w = w;
+    p.seq_lens = pc.seq_lens;
+    p.page_table = pc.page_table;
+    p.page_size = pc.page_size;
+    p.max_pages = pc.max_pages;
+    p.num_pages = pc.num_pages;
     p.B = B;
     p.q_pos0 = q_pos0;
     p.n_kv = n_kv;
@@ -356,7 +409,7 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
 }
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms) {
-    const int nkt = (q_pos0 + 1 + 127) / 128;
+    const int nkt = (q_pos0 + 1 + 127) / 128;  // paged: q_pos0 = the longest sequence - 1
     int splits = dec_splits(B, nkt, num_sms);
     const int tps = (nkt + splits - 1) / splits;
     splits = (nkt + tps - 1) / tps;
@@ -365,8 +418,19 @@ size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms) 
 
 cudaError_t launch_indexer_decode(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int H,
                                   int topk, int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
-    if (H == 32) return launch_dec_t<32>(q, k, w, B, q_pos0, n_kv, topk, idx_out, ws, num_sms, stream);
-    if (H == 64) return launch_dec_t<64>(q, k, w, B, q_pos0, n_kv, topk, idx_out, ws, num_sms, stream);
+    const DecCache none = {nullptr, nullptr, 0, 0, 0, 0};
+    if (H == 32) return launch_dec_t<32>(q, k, w, B, q_pos0, n_kv, topk, none, idx_out, ws, num_sms, stream);
+    if (H == 64) return launch_dec_t<64>(q, k, w, B, q_pos0, n_kv, topk, none, idx_out, ws, num_sms, stream);
+    return cudaErrorNotSupported;
+}
+
+cudaError_t launch_indexer_decode_paged(const void* q, const void* k_pages, const int* page_table, const int* seq_lens,
+                                        const float* w, int B, int max_len, int page_size, int num_pages,
+                                        int max_pages, int H, int topk, int* idx_out, void* ws, int num_sms,
+                                        cudaStream_t stream) {
+    const DecCache pc = {seq_lens, page_table, page_size, max_pages, num_pages, max_len};
+    if (H == 32) return launch_dec_t<32>(q, k_pages, w, B, max_len - 1, 0, topk, pc, idx_out, ws, num_sms, stream);
+    if (H == 64) return launch_dec_t<64>(q, k_pages, w, B, max_len - 1, 0, topk, pc, idx_out, ws, num_sms, stream);
     return cudaErrorNotSupported;
 }
 

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(WARPS * 32)
                        const __nv_bfloat16* __restrict__ V, const int* __restrict__ idx, int B, int n_q,
                        int n_kv, int Hq, int Hkv, int topk, float scale_log2, void* __restrict__ O,
                        int splits, int chunks_per_split, float* __restrict__ part, IdxShare share,
-                       WsHeader* hdr) {
+                       KvPages pg, WsHeader* hdr) {
     using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,18 +126,30 @@ __global__ void __launch_bounds__(WARPS * 32)
         const int qi = static_cast<int>(row - b * n_q);
         const int* irow = idx + (b * share.rows(n_q) + qi / share.q_per_idx) * topk;
         const int lim = share.limit(qi);  // shared rows: keys past this query's own position are skipped
-        const __nv_bfloat16* kb = K + static_cast<size_t>(b) * n_kv * tok_stride + static_cast<size_t>(g) * D;
-        const __nv_bfloat16* vb = V + static_cast<size_t>(b) * n_kv * tok_stride + static_cast<size_t>(g) * D;
+        const size_t seq_off = pg.table ? 0 : static_cast<size_t>(b) * n_kv * tok_stride;
+        const __nv_bfloat16* kb = K + seq_off + static_cast<size_t>(g) * D;
+        const __nv_bfloat16* vb = V + seq_off + static_cast<size_t>(g) * D;
+        const int n_valid = pg.lens ? min(__ldg(pg.lens + b), pg.max_pages * pg.page_size) : n_kv;
 
-        // index of key `lane` of chunk c (-1 past the end); out-of-range entries are flagged and skipped
+        // cache row of key `lane` of chunk c (-1 past the end); out-of-range entries are flagged and skipped
         auto load_idx = [&](int c) -> int {
             const int kk = c * CHUNK + lane;
             int t = (lane < CHUNK && kk < topk) ? __ldg(irow + kk) : -1;
-            if (t < -1 || t >= n_kv) {
+            if (t < -1 || t >= n_valid) {
                 raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
                 t = -1;
             }
-            return t > lim ? -1 : t;
+            if (t > lim) t = -1;
+            if (pg.table && t >= 0) {
+                const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + t / pg.page_size);
+                if (page < 0 || page >= pg.num_pages) {
+                    raise_status(hdr, DSA_STATUS_BAD_INDEX, page);
+                    t = -1;
+                } else {
+                    t = page * pg.page_size + t % pg.page_size;
+                }
+            }
+            return t;
         };
         // gather chunk c's K and V slices into stage c % STAGES (always commits one group)
         auto issue = [&](int c, int tsel) {
@@ -391,7 +403,7 @@ static int attn_splits(long long units, int nchunks, int warps, int num_sms, int
 template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ = false, bool QK_SPLIT = false>
 static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                                  const int* idx, int B, int n_q, int n_kv, int Hq, int Hkv, int topk,
-                                 float scale, void* O, bool out_bf16, IdxShare share, WsHeader* hdr,
+                                 float scale, void* O, bool out_bf16, IdxShare share, KvPages pg, WsHeader* hdr,
                                  int num_sms, cudaStream_t stream) {
     using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
     auto kern = out_bf16 ? sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, true>
@@ -413,7 +425,7 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
     const float scale_log2 = scale * 1.4426950408889634f;
     float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(hdr) + kWsHeaderBytes);
     kern<<<static_cast<int>(grid), WARPS * 32, C::SMEM, stream>>>(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, topk,
-                                                                   scale_log2, O, splits, per, part, share, hdr);
+                                                                   scale_log2, O, splits, per, part, share, pg, hdr);
     if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
     const int G = Hq / Hkv;
     dim3 mg(static_cast<unsigned>(units), static_cast<unsigned>(G));
@@ -438,7 +450,7 @@ size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, 
 // Host dispatcher: returns cudaErrorNotSupported for shapes without a kernel.
 cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, const int* idx, int B, int n_q,
                                int n_kv, int Hq, int Hkv, int d, int topk, float scale, void* O, bool out_bf16,
-                               IdxShare share, WsHeader* hdr, int num_sms, cudaStream_t stream) {
+                               IdxShare share, KvPages pg, WsHeader* hdr, int num_sms, cudaStream_t stream) {
     auto q = static_cast<const __nv_bfloat16*>(Q);
     auto k = static_cast<const __nv_bfloat16*>(K);
     auto v = static_cast<const __nv_bfloat16*>(V);
@@ -446,10 +458,10 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
     // holds (measured on B200: warps in flight matter more than stages per warp).
     if (d == 128)
         return launch_attn_t<128, 16, 2, kAttnWarpsD128, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
-                                                         out_bf16, share, hdr, num_sms, stream);
+                                                         out_bf16, share, pg, hdr, num_sms, stream);
     if (d == 64)
         return launch_attn_t<64, 16, 2, kAttnWarpsD64, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
-                                                        out_bf16, share, hdr, num_sms, stream);
+                                                        out_bf16, share, pg, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }
 

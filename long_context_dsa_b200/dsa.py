@@ -29,6 +29,7 @@ ABI_SYMBOLS = (
     "sparse_attn_topk_workspace_size", "sparse_attn_topk", "sparse_attn_topk_shared",
     "layer_group_forward_workspace_size", "layer_group_forward",
     "idx_score_topk_noalloc", "idx_overlap", "layer_pattern_search",
+    "idx_score_topk_paged_workspace_size", "idx_score_topk_paged", "sparse_attn_topk_paged",
 )
 
 
@@ -92,6 +93,9 @@ def lib() -> ctypes.CDLL:
                                  ctypes.POINTER(IndexCacheStruct), ctypes.POINTER(GroupStats), vp, sz, vp], i),
         "idx_score_topk_noalloc": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp], i),
         "idx_overlap": ([vp, vp, i64, i, vp, vp], i),
+        "idx_score_topk_paged_workspace_size": ([i, i, i, i, i, psz], i),
+        "idx_score_topk_paged": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp, sz, vp], i),
+        "sparse_attn_topk_paged": ([vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, i, vp, sz, vp], i),
         "layer_pattern_search": ([ctypes.POINTER(ctypes.c_double), i, i, ctypes.c_char_p], i),
     }
     for name, (args, res) in sig.items():
@@ -315,6 +319,62 @@ def sparse_attn_topk_shared(Q, K, V, idx, q_per_idx: int, q_pos0: int, scale: fl
     _check(lib().sparse_attn_topk_shared(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), B, n_q, q_pos0, n_kv, Hq, Hkv, d_qk,
                                          d_v, topk, q_per_idx, float(scale or 0.0), _ptr(out), od, _ptr(workspace),
                                          workspace.numel(), _stream(stream)))
+    return out
+
+
+# -------------------------------------------------------------- paged decode
+def idx_score_topk_paged(q_I, k_pages, page_table, seq_lens, w, topk: int, max_seq_len: int, out=None,
+                         workspace=None, stream=None) -> torch.Tensor:
+    """One query per sequence over a paged key cache: q_I [B, H, d], k_pages [num_pages, page_size, d],
+    page_table [B, max_pages], seq_lens [B] (int32, device) -> idx [B, topk]."""
+    _need(q_I, torch.bfloat16, "q_I")
+    _need(k_pages, torch.bfloat16, "k_pages")
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    _need(w, torch.float32, "w")
+    B, H, d = q_I.shape
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    max_pages = page_table.shape[1]
+    if out is None:
+        out = torch.empty((B, topk), dtype=torch.int32, device=q_I.device)
+    if workspace is None:
+        n = ctypes.c_size_t(0)
+        _check(lib().idx_score_topk_paged_workspace_size(B, max_seq_len, H, d, topk, ctypes.byref(n)))
+        workspace = _workspace(n.value, q_I.device)
+    _check(lib().idx_score_topk_paged(_ptr(q_I), _ptr(k_pages), _ptr(page_table), _ptr(seq_lens), _ptr(w), B,
+                                      max_seq_len, page_size, num_pages, max_pages, H, d, topk, _ptr(out),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def idx_score_topk_paged_workspace_size(B, max_seq_len, H, d, topk) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().idx_score_topk_paged_workspace_size(B, max_seq_len, H, d, topk, ctypes.byref(n)))
+    return n.value
+
+
+def sparse_attn_topk_paged(Q, K_pages, V_pages, page_table, seq_lens, idx, scale: float | None = None,
+                           o_dtype=torch.float32, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """Q [B, Hq, d]; K_pages, V_pages [num_pages, page_size, Hkv, d]; idx [B, topk] -> O [B, Hq, d]."""
+    for t, n in ((Q, "Q"), (K_pages, "K_pages"), (V_pages, "V_pages")):
+        _need(t, torch.bfloat16, n)
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    _need(idx, torch.int32, "idx")
+    B, Hq, d = Q.shape
+    num_pages, page_size, Hkv = K_pages.shape[0], K_pages.shape[1], K_pages.shape[2]
+    max_pages = page_table.shape[1]
+    topk = idx.shape[-1]
+    od = DSA_F32 if o_dtype == torch.float32 else DSA_BF16
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=o_dtype, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(sparse_attn_topk_workspace_size(B, 1, num_pages * page_size, Hq, Hkv, d, d, topk),
+                               Q.device)
+    _check(lib().sparse_attn_topk_paged(_ptr(Q), _ptr(K_pages), _ptr(V_pages), _ptr(page_table), _ptr(seq_lens),
+                                        _ptr(idx), B, page_size, num_pages, max_pages, Hq, Hkv, d, topk,
+                                        float(scale or 0.0), _ptr(out), od, _ptr(workspace), workspace.numel(),
+                                        _stream(stream)))
     return out
 
 

@@ -26,4 +26,5 @@ from .dsa_oracle import (  # noqa: F401
     overlap_counts,
     pattern_loss,
     pattern_search,
+    gather_paged,
 )

@@ -383,3 +383,15 @@ def pattern_search(overlap, n_f: int) -> str:
                 best, best_loss = l, loss
         pat[best] = "S"
     return "".join(pat)
+
+
+# ---------------------------------------------------------------------------
+# paged caches (serving layout)
+# ---------------------------------------------------------------------------
+
+def gather_paged(pool, page_table_row, length: int, page_size: int) -> np.ndarray:
+    """Logical cache [length, ...] of one sequence from a page pool [num_pages * page_size, ...]:
+    token t sits in row page_table_row[t // page_size] * page_size + t % page_size."""
+    pool = np.asarray(pool)
+    rows = [int(page_table_row[t // page_size]) * page_size + t % page_size for t in range(length)]
+    return pool[rows]

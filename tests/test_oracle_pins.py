@@ -410,6 +410,22 @@ def test_pattern_search_finds_segment_starts_and_the_optimum():
     assert oracle.pattern_loss(ov, got) == pytest.approx(oracle.pattern_loss(ov, best))
 
 
+def test_gather_paged_identity_and_scatter_round_trip():
+    rng = np.random.default_rng(19)
+    P, n = 4, 10
+    seq = rng.standard_normal((n, 3))
+    # identity table over a pool that is the sequence itself (padded to whole pages)
+    pool = np.concatenate([seq, np.zeros((2, 3))])
+    assert np.array_equal(oracle.gather_paged(pool, [0, 1, 2], n, P), seq)
+    # scattered into shuffled pages of a larger pool, gathered back
+    perm = [5, 2, 7]
+    big = np.full((8 * P, 3), np.nan)
+    for lp, pp in enumerate(perm):
+        chunk = seq[lp * P:(lp + 1) * P]
+        big[pp * P:pp * P + len(chunk)] = chunk
+    assert np.array_equal(oracle.gather_paged(big, perm + [-1, -1], n, P), seq)
+
+
 @pytest.mark.parametrize("bad", ["", "S", "SFFF", "FXS", "fsss"])
 def test_pattern_rejects(bad):
     with pytest.raises(ValueError):
