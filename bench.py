@@ -602,14 +602,15 @@ def run_paged(args, dev):
     seq = torch.from_numpy(lens).to(dev)
     idx = torch.empty((B, TOPK), dtype=torch.int32, device=dev)
     O = torch.empty((B, HQ, DH), dtype=torch.bfloat16, device=dev)
-    ws = torch.zeros(max(dsa.idx_score_topk_paged_workspace_size(B, Lmax, H_I, D_I, TOPK),
+    max_len = int(lens.max())
+    ws = torch.zeros(max(dsa.idx_score_topk_paged_workspace_size(B, max_len, H_I, D_I, TOPK),
                          dsa.sparse_attn_topk_workspace_size(B, 1, num_pages * P, HQ, HKV, DH, DH, TOPK)),
                      dtype=torch.uint8, device=dev)
 
     def step(evs=None):
         if evs:
             evs[0].record()
-        dsa.idx_score_topk_paged(q, k_pool, table, seq, w, TOPK, Lmax, out=idx, workspace=ws)
+        dsa.idx_score_topk_paged(q, k_pool, table, seq, w, TOPK, max_len, out=idx, workspace=ws)
         if evs:
             evs[1].record()
         for (Q, Kp, Vp) in layers:
