@@ -22,7 +22,7 @@ cudaError_t launch_indexer_decode_paged(const void* q, const void* k_pages, cons
                                         const float* w, int B, int max_len, int page_size, int num_pages,
                                         int max_pages, int H, int topk, int* idx_out, void* ws, int num_sms,
                                         cudaStream_t stream);
-size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms);
+size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen);
 cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
                                       int Hq, int topk, float scale, void* O, bool out_bf16, IdxShare share,
                                       WsHeader* hdr, int num_sms, cudaStream_t stream);
@@ -382,7 +382,7 @@ int idx_score_topk_paged_workspace_size(int B, int max_seq_len, int H_I, int d_I
     int sms;
     int rc = sm_count(&sms);
     if (rc) return rc;
-    *bytes = kWsHeaderBytes + indexer_decode_workspace_bytes(B, max_seq_len - 1, topk, sms);
+    *bytes = kWsHeaderBytes + indexer_decode_workspace_bytes(B, max_seq_len - 1, topk, sms, true);
     return DSA_OK;
 }
 

@@ -518,14 +518,14 @@ cudaError_t launch_t(const void* q, const float* q_scale, const void* k, const f
 }  // namespace
 
 bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype);
-size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms);
+size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen);
 cudaError_t launch_indexer_decode(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int H,
                                   int topk, int* idx_out, void* ws, int num_sms, cudaStream_t stream);
 
 size_t indexer_workspace_bytes(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype,
                                int num_sms) {
     if (indexer_decode_supported(B, n_q, q_pos0, n_kv, H, d, topk, dtype))
-        return indexer_decode_workspace_bytes(B, q_pos0, topk, num_sms);
+        return indexer_decode_workspace_bytes(B, q_pos0, topk, num_sms, false);
     const int n_tiles = tiles_per_b(n_q, H) * B;
     const int grid = grid_for(n_tiles, num_sms);
     const size_t qg = 256 / H;
