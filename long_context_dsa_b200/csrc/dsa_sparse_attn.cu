@@ -85,48 +85,13 @@ struct AttnCfg {
     }
 };
 
-// Combine the `splits` ranges of one (query row, KV head) unit with one warp:
-// per query head, O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s
-// (ranges that saw no key have m_s = -inf and drop out).  pu: the unit's
-// [splits][G][D + 2] partial state; out_off: element offset of its G heads in O.
-template <int D, bool OUT_BF16>
-__device__ __noinline__ void merge_unit(const float* pu, int G, int splits, int lane, void* O, size_t out_off) {
-    const size_t sstride = static_cast<size_t>(G) * (D + 2);
-    for (int h = 0; h < G; ++h) {
-        const float* ph = pu + h * (D + 2);
-        float M = -INFINITY;
-        for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(ph + s * sstride + D));
-        float L = 0.f;
-        float acc[D / 32];
-#pragma unroll
-        for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            const float m = __ldcg(ph + s * sstride + D);
-            if (m == -INFINITY) continue;
-            const float f = exp2f(m - M);
-            L += f * __ldcg(ph + s * sstride + D + 1);
-#pragma unroll
-            for (int i = 0; i < D / 32; ++i) acc[i] += f * __ldcg(ph + s * sstride + i * 32 + lane);
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int i = 0; i < D / 32; ++i) {
-            const size_t o = out_off + static_cast<size_t>(h) * D + i * 32 + lane;
-            if (OUT_BF16)
-                reinterpret_cast<__nv_bfloat16*>(O)[o] = __float2bfloat16_rn(acc[i] * inv);
-            else
-                reinterpret_cast<float*>(O)[o] = acc[i] * inv;
-        }
-    }
-}
-
 template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ, bool QK_SPLIT, bool OUT_BF16>
 __global__ void __launch_bounds__(WARPS * 32)
     sparse_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                        const __nv_bfloat16* __restrict__ V, const int* __restrict__ idx, int B, int n_q,
                        int n_kv, int Hq, int Hkv, int topk, float scale_log2, void* __restrict__ O,
-                       int splits, int chunks_per_split, float* __restrict__ part, int* __restrict__ done,
-                       IdxShare share, KvPages pg, WsHeader* hdr) {
+                       int splits, int chunks_per_split, float* __restrict__ part, IdxShare share,
+                       KvPages pg, WsHeader* hdr) {
     using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,8 +101,7 @@ __global__ void __launch_bounds__(WARPS * 32)
 
     const int G = Hq / Hkv;
     // work items: (query row, KV head) units, each cut into `splits` ranges of chunks; with
-    // splits > 1 a warp writes its range's softmax state to `part`, and the warp that finishes
-    // a unit's last range combines them (merge_unit)
+    // splits > 1 a warp writes its range's softmax state to `part` and attn_merge_kernel combines
     const long long units = static_cast<long long>(B) * n_q * Hkv;
     const long long items = units * splits;
     const int nchunks = (topk + CHUNK - 1) / CHUNK;
@@ -356,18 +320,6 @@ __global__ void __launch_bounds__(WARPS * 32)
                     }
                 }
             }
-            // the warp that completes a unit's last range combines all ranges of the unit
-            // (stores, then a device-scope fence, then the count: the classic last-block pattern)
-            __threadfence();
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) last = atomicAdd(done + u, 1) == splits - 1;
-            if (__shfl_sync(0xffffffffu, last, 0)) {
-                __threadfence();
-                merge_unit<D, OUT_BF16>(part + static_cast<size_t>(u) * splits * G * (D + 2), G, splits, lane,
-                                        O, (static_cast<size_t>(row) * Hq + static_cast<size_t>(g) * G) * D);
-                if (lane == 0) done[u] = 0;  // ready for the next launch
-            }
             continue;
         }
         const float inv0 = lrun[0] > 0.f ? 1.f / lrun[0] : 0.f;
@@ -393,6 +345,39 @@ __global__ void __launch_bounds__(WARPS * 32)
                 }
             }
         }
+    }
+}
+
+// Combine the split ranges of each (query row, KV head, query head):
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.
+template <bool OUT_BF16>
+__global__ void attn_merge_kernel(const float* __restrict__ part, int G, int D, int splits, int Hq, int Hkv,
+                                  void* __restrict__ O) {
+    const long long u = blockIdx.x;  // (row, g)
+    const int h = blockIdx.y;
+    const long long row = u / Hkv;
+    const int g = static_cast<int>(u % Hkv);
+    const float* p0 = part + (static_cast<size_t>(u) * splits * G + h) * (D + 2);
+    const size_t sstride = static_cast<size_t>(G) * (D + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, p0[s * sstride + D]);
+    float L = 0.f;
+    for (int s = 0; s < splits; ++s) {
+        const float m = p0[s * sstride + D];
+        L += (m == -INFINITY) ? 0.f : exp2f(m - M) * p0[s * sstride + D + 1];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float m = p0[s * sstride + D];
+            if (m != -INFINITY) acc += exp2f(m - M) * p0[s * sstride + d];
+        }
+        const size_t ob = (static_cast<size_t>(row) * Hq + g * G + h) * D + d;
+        if (OUT_BF16)
+            reinterpret_cast<__nv_bfloat16*>(O)[ob] = __float2bfloat16_rn(acc * inv);
+        else
+            reinterpret_cast<float*>(O)[ob] = acc * inv;
     }
 }
 
@@ -439,13 +424,15 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
     if (grid < 1) grid = 1;
     const float scale_log2 = scale * 1.4426950408889634f;
     float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(hdr) + kWsHeaderBytes);
-    const int G = Hq / Hkv;
-    int* done = reinterpret_cast<int*>(part + static_cast<size_t>(units) * splits * G * (D + 2));
-    if (splits > 1 && (e = cudaMemsetAsync(done, 0, static_cast<size_t>(units) * sizeof(int), stream)) != cudaSuccess)
-        return e;
     kern<<<static_cast<int>(grid), WARPS * 32, C::SMEM, stream>>>(Q, K, V, idx, B, n_q, n_kv, Hq, Hkv, topk,
-                                                                   scale_log2, O, splits, per, part, done, share, pg,
-                                                                   hdr);
+                                                                   scale_log2, O, splits, per, part, share, pg, hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    const int G = Hq / Hkv;
+    dim3 mg(static_cast<unsigned>(units), static_cast<unsigned>(G));
+    if (out_bf16)
+        attn_merge_kernel<true><<<mg, 128, 0, stream>>>(part, G, D, splits, Hq, Hkv, O);
+    else
+        attn_merge_kernel<false><<<mg, 128, 0, stream>>>(part, G, D, splits, Hq, Hkv, O);
     return cudaGetLastError();
 }
 
@@ -457,9 +444,7 @@ size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, 
     int per = 0;
     const int splits = attn_splits(units, (topk + 15) / 16, warps, num_sms, &per);
     if (splits == 1) return 0;
-    // partial state of every (unit, range), then one completion count per unit
-    return static_cast<size_t>(units) * splits * (Hq / Hkv) * (d + 2) * sizeof(float) +
-           static_cast<size_t>(units) * sizeof(int);
+    return static_cast<size_t>(units) * splits * (Hq / Hkv) * (d + 2) * sizeof(float);
 }
 
 // Host dispatcher: returns cudaErrorNotSupported for shapes without a kernel.
