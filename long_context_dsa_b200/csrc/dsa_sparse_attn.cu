@@ -85,7 +85,11 @@ struct AttnCfg {
     }
 };
 
-template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ, bool QK_SPLIT, bool OUT_BF16>
+// Compile-time switches, so the plain path carries none of the bookkeeping of the others:
+// SPLIT: units cut into index ranges (few rows, e.g. decode); PAGED: K/V in a page pool;
+// SHARED: query rows share index rows.
+template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ, bool QK_SPLIT, bool OUT_BF16, bool SPLIT, bool PAGED,
+          bool SHARED>
 __global__ void __launch_bounds__(WARPS * 32)
     sparse_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                        const __nv_bfloat16* __restrict__ V, const int* __restrict__ idx, int B, int n_q,
@@ -103,7 +107,7 @@ __global__ void __launch_bounds__(WARPS * 32)
     // work items: (query row, KV head) units, each cut into `splits` ranges of chunks; with
     // splits > 1 a warp writes its range's softmax state to `part` and attn_merge_kernel combines
     const long long units = static_cast<long long>(B) * n_q * Hkv;
-    const long long items = units * splits;
+    const long long items = SPLIT ? units * splits : units;
     const int nchunks = (topk + CHUNK - 1) / CHUNK;
     const size_t tok_stride = static_cast<size_t>(Hkv) * D;  // elements per token row of K / V
 
@@ -116,20 +120,20 @@ __global__ void __launch_bounds__(WARPS * 32)
 
     for (long long it = static_cast<long long>(blockIdx.x) * WARPS + warp; it < items;
          it += static_cast<long long>(gridDim.x) * WARPS) {
-        const long long u = it / splits;
-        const int sp = static_cast<int>(it % splits);
-        const int c0 = sp * chunks_per_split;
-        const int c1 = min(nchunks, c0 + chunks_per_split);
+        const long long u = SPLIT ? it / splits : it;
+        const int sp = SPLIT ? static_cast<int>(it % splits) : 0;
+        const int c0 = SPLIT ? sp * chunks_per_split : 0;
+        const int c1 = SPLIT ? min(nchunks, c0 + chunks_per_split) : nchunks;
         const long long row = u / Hkv;
         const int g = static_cast<int>(u % Hkv);
         const long long b = row / n_q;
         const int qi = static_cast<int>(row - b * n_q);
-        const int* irow = idx + (b * share.rows(n_q) + qi / share.q_per_idx) * topk;
-        const int lim = share.limit(qi);  // shared rows: keys past this query's own position are skipped
-        const size_t seq_off = pg.table ? 0 : static_cast<size_t>(b) * n_kv * tok_stride;
+        const int* irow = SHARED ? idx + (b * share.rows(n_q) + qi / share.q_per_idx) * topk : idx + row * topk;
+        const int lim = SHARED ? share.limit(qi) : 0;  // shared rows: keys past the query's own position are skipped
+        const size_t seq_off = PAGED ? 0 : static_cast<size_t>(b) * n_kv * tok_stride;
         const __nv_bfloat16* kb = K + seq_off + static_cast<size_t>(g) * D;
         const __nv_bfloat16* vb = V + seq_off + static_cast<size_t>(g) * D;
-        const int n_valid = pg.lens ? min(__ldg(pg.lens + b), pg.max_pages * pg.page_size) : n_kv;
+        const int n_valid = PAGED ? min(__ldg(pg.lens + b), pg.max_pages * pg.page_size) : n_kv;
 
         // cache row of key `lane` of chunk c (-1 past the end); out-of-range entries are flagged and skipped
         auto load_idx = [&](int c) -> int {
@@ -139,8 +143,8 @@ __global__ void __launch_bounds__(WARPS * 32)
                 raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
                 t = -1;
             }
-            if (t > lim) t = -1;
-            if (pg.table && t >= 0) {
+            if (SHARED && t > lim) t = -1;
+            if (PAGED && t >= 0) {
                 const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + t / pg.page_size);
                 if (page < 0 || page >= pg.num_pages) {
                     raise_status(hdr, DSA_STATUS_BAD_INDEX, page);
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(WARPS * 32)
         // gather chunk c's K and V slices into stage c % STAGES (always commits one group)
         auto issue = [&](int c, int tsel) {
             if (c < c1) {
-                const int s = (c - c0) % STAGES;
+                const int s = (SPLIT ? c - c0 : c) % STAGES;
                 if (lane < CHUNK) sidx[s * CHUNK + lane] = tsel;
                 const uint32_t kst = ring_s + s * C::STAGE_BYTES;
                 const uint32_t vst = kst + CHUNK * C::RS;
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(WARPS * 32)
             t_next = load_idx(c + STAGES);
             cp_async_wait<STAGES - 1>();
             __syncwarp();
-            const int s = (c - c0) % STAGES;
+            const int s = (SPLIT ? c - c0 : c) % STAGES;
             const uint32_t kst = ring_s + s * C::STAGE_BYTES;
             const uint32_t vst = kst + CHUNK * C::RS;
             const int* si = sidx + s * CHUNK;
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) lrun[j] += __shfl_xor_sync(0xffffffffu, lrun[j], off);
         }
-        if (splits > 1) {
+        if (SPLIT) {
             // this range's state per head: unnormalised O, running max (log2 units), sum
             float* pb = part + static_cast<size_t>(it) * G * (D + 2);
 #pragma unroll
@@ -406,18 +410,28 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
                                  float scale, void* O, bool out_bf16, IdxShare share, KvPages pg, WsHeader* hdr,
                                  int num_sms, cudaStream_t stream) {
     using C = AttnCfg<D, CHUNK, STAGES, WARPS, SWZ>;
-    auto kern = out_bf16 ? sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, true>
-                         : sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, false>;
+    const long long units = static_cast<long long>(B) * n_q * Hkv;
+    const int nchunks = (topk + CHUNK - 1) / CHUNK;
+    int per = nchunks;
+    const int splits = attn_splits(units, nchunks, WARPS, num_sms, &per);
+    using KernFn = void (*)(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*, const int*, int, int, int,
+                            int, int, int, float, void*, int, int, float*, IdxShare, KvPages, WsHeader*);
+    // (out_bf16, split, paged, shared); paged and shared never combine in the API
+#define DSA_K(OB, SP, PG, SH) sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, OB, SP, PG, SH>
+    static const KernFn table[2][2][3] = {
+        {{DSA_K(false, false, false, false), DSA_K(false, false, true, false), DSA_K(false, false, false, true)},
+         {DSA_K(false, true, false, false), DSA_K(false, true, true, false), DSA_K(false, true, false, true)}},
+        {{DSA_K(true, false, false, false), DSA_K(true, false, true, false), DSA_K(true, false, false, true)},
+         {DSA_K(true, true, false, false), DSA_K(true, true, true, false), DSA_K(true, true, false, true)}}};
+#undef DSA_K
+    const int mode = pg.table ? 1 : (share.q_per_idx > 1 || share.causal) ? 2 : 0;
+    KernFn kern = table[out_bf16 ? 1 : 0][splits > 1 ? 1 : 0][mode];
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
     if (e != cudaSuccess) return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, C::SMEM);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
-    const long long units = static_cast<long long>(B) * n_q * Hkv;
-    const int nchunks = (topk + CHUNK - 1) / CHUNK;
-    int per = nchunks;
-    const int splits = attn_splits(units, nchunks, WARPS, num_sms, &per);
     long long grid = static_cast<long long>(num_sms) * per_sm;
     const long long need = (units * splits + WARPS - 1) / WARPS;
     if (grid > need) grid = need;
