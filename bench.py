@@ -107,6 +107,24 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
+def adjacent_overlap(layers, dev, rows=2048):
+    """Mean top-k overlap of adjacent layers' own selections (the pages report 70-100%) over the
+    last `rows` query rows: each layer's indexer runs on them alone, idx_overlap counts the
+    shared indices."""
+    import torch
+    from long_context_dsa_b200 import dsa
+
+    p0 = L - rows
+    sel = []
+    for Lh in layers[:4]:
+        sel.append(dsa.idx_score_topk(Lh["q_I"][:, p0:].contiguous(), Lh["k_I"], Lh["w"][:, p0:].contiguous(),
+                                      TOPK, q_pos0=p0))
+    fr = [float(dsa.idx_overlap(sel[l], sel[l + 1]).double().mean().item()) / TOPK for l in range(len(sel) - 1)]
+    torch.cuda.synchronize()
+    return {"rows": f"last {rows} of {L}", "layers": "0-1, 1-2, 2-3", "values": [round(x, 4) for x in fr],
+            "mean": round(sum(fr) / len(fr), 4)}
+
+
 def attn_traffic():
     """DRAM bytes of one full sparse-attention launch, scaled from the ncu capture of the tail case
     (4096 rows x 2048 selected keys: 2.539 GB read + 0.037 GB written) by selected (query, key) pairs;
@@ -185,6 +203,7 @@ def run_gpu(args, rank, world, local_rank):
     dsa.check_status(ws)
     allf_idx = [allf_evs[3 * l].elapsed_time(allf_evs[3 * l + 1]) for l in range(N_LAYERS)]
     allf_step = allf_evs[0].elapsed_time(allf_evs[-1])
+    overlap = adjacent_overlap(layers, dev)
 
     # ---- end to end through the public API from pinned host memory
     e2e = None
@@ -231,7 +250,8 @@ def run_gpu(args, rank, world, local_rank):
         "index_sharing": {"all_f_step_ms": round(allf_step, 3), "shared_step_ms": round(ms_per_step, 3),
                           "all_f_indexer_ms": round(sum(allf_idx), 3),
                           "shared_indexer_ms": round(sum(idx_ms) / args.steps, 3),
-                          "indexer_time_ratio": round(sum(allf_idx) / (sum(idx_ms) / args.steps), 3)},
+                          "indexer_time_ratio": round(sum(allf_idx) / (sum(idx_ms) / args.steps), 3),
+                          "adjacent_layer_overlap": overlap},
         "gpu_launches": launches,
         "clocks": clocks,
     }
@@ -485,6 +505,53 @@ def run_decode(args, dev):
             "all_f_tok_per_s": round(B / (res["FFFF"][0] / 1e3), 1)}
 
 
+def run_decode_mha(args, dev):
+    """Decode with 32 KV heads (MHA, the config's head count) at B = 8: the 200K cache of 64 such
+    sequences would not fit one GPU (210 GB per layer).  4 layers FSSS, top-2048."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    B, Lc, Hkv = 8, 200000, 32
+    gen = synth.StructuredIndexer("decodemha", B, Lc, H_I, D_I, r=32, base_std=1.0, noise_std=0.2, device=dev,
+                                  seed=5000)
+    layers = []
+    for l in range(4):
+        Lh = {}
+        Lh["q_I"], Lh["w"] = gen.queries(l, Lc - 1, Lc)
+        Lh["k_I"] = gen.keys(l)
+        Lh["Q"], Lh["K"], Lh["V"] = synth.attention_inputs("decodemha", l, B, 1, Lc, HQ, Hkv, DH, DH, device=dev,
+                                                           seed=5000)
+        Lh["O"] = torch.empty((B, 1, HQ, DH), dtype=torch.bfloat16, device=dev)
+        layers.append(Lh)
+    del gen
+    shape = dsa.group_shape(B, 1, Lc - 1, Lc, H_I, D_I, HQ, Hkv, DH, DH, TOPK, o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((B, 1, TOPK), dtype=torch.int32, device=dev))
+    for _ in range(3):
+        dsa.layer_group_forward(shape, layers, "FSSS", cache, workspace=ws)
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(12)]
+    for e in evs:
+        e.record()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 10
+    a.record()
+    for i in range(n):
+        dsa.layer_group_forward(shape, layers, "FSSS", cache, workspace=ws, events=evs if i == n - 1 else None)
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b) / n
+    att_ms = sum(evs[3 * l + 1].elapsed_time(evs[3 * l + 2]) for l in range(4))
+    abytes = B * TOPK * Hkv * 2 * DH * 2
+    del layers
+    torch.cuda.empty_cache()
+    return {"workload": f"decode B={B} at a {Lc}-token cache, 4 layers FSSS, MHA {HQ}Q/{Hkv}KV d={DH}, top-{TOPK}",
+            "tok_per_s": round(B / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "attention_ms": round(att_ms, 4),
+            "attention_gathered_gbs": round(4 * abytes / (att_ms / 1e3) / 1e9, 1)}
+
+
 def run_mtp(args, dev):
     """Multi-token (speculative) decode: 64 sequences verify 4 draft tokens each at a 200000-token
     cache, 4 layers FSSS.  Shared: the F layer selects once, for the last draft token, and all 4
@@ -696,6 +763,9 @@ def run_ctx1m(args, dev):
             "chunk_ms": round(ms, 3), "chunk_tok_per_s": round(C / (ms / 1e3), 1),
             "indexer_ms_per_f_layer": round(idx_avg, 3),
             "indexer_fp8_tflops": round(iflops / (idx_avg / 1e3) / 1e12, 1),
+            # no measured fp8 peak: the measured sustained bf16 peak x the nominal fp8/bf16 ratio (4.5/2.25)
+            "indexer_fp8_frac": round(iflops / (idx_avg / 1e3) / 1e12 / (2 * peaks()[2]), 4),
+            "indexer_fp8_peak_source": "2 x measured bf16_tflops_sustained (nominal fp8/bf16 ratio)",
             "attention_ms_per_layer": round(sum(att_ms) / len(att_ms), 3),
             "attention_gathered_gbs": round(abytes / (sum(att_ms) / len(att_ms) / 1e3) / 1e9, 1),
             "full_prefill_estimate_s": round(est_s, 2),
@@ -712,17 +782,18 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
-    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "ctx1m", "mtp", "paged"],
+    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m: only that "
                          "extra measurement, printed as one JSON line")
     args = ap.parse_args()
     if args.case == "profile":
         run_profile_case(args)
         return
-    if args.case in ("decode", "ctx1m", "mtp", "paged"):
+    if args.case in ("decode", "decode_mha", "ctx1m", "mtp", "paged"):
         import torch
         dev = torch.device("cuda", 0)
-        fn = {"decode": run_decode, "ctx1m": run_ctx1m, "mtp": run_mtp, "paged": run_paged}[args.case]
+        fn = {"decode": run_decode, "decode_mha": run_decode_mha, "ctx1m": run_ctx1m, "mtp": run_mtp,
+              "paged": run_paged}[args.case]
         print(json.dumps({"case": args.case, **fn(args, dev)}), flush=True)
         return
 
@@ -754,6 +825,7 @@ def main():
         torch.cuda.empty_cache()
         dev = torch.device("cuda", local_rank)
         out["decode"] = run_decode(args, dev)
+        out["decode_mha32_b8"] = run_decode_mha(args, dev)
         out["multi_token_decode"] = run_mtp(args, dev)
         out["paged_decode"] = run_paged(args, dev)
         out["context_1m_tail_chunk"] = run_ctx1m(args, dev)
