@@ -806,7 +806,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
-    ap.add_argument("--case", default="bench", choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged"],
+    ap.add_argument("--case", default="bench",
+                    choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m: only that "
                          "extra measurement, printed as one JSON line")
     args = ap.parse_args()
