@@ -28,7 +28,7 @@
 namespace dsa {
 
 cudaError_t launch_topk_merge_pairs(const uint32_t* keys, const int* idxs, int rows, int len, int k, int* out,
-                                    WsHeader* hdr, int num_sms, cudaStream_t stream);
+                                    WsHeader* hdr, int num_sms, cudaStream_t stream, int n_tok);
 
 template <int H>
 struct DecCfg {
@@ -399,7 +399,7 @@ cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, in
     kern<<<units < num_sms ? units : num_sms, C::THREADS, C::SMEM, stream>>>(mq, mk, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return launch_topk_merge_pairs(p.part_key, p.part_idx, B, p.splits * topk, topk, idx_out, p.hdr, num_sms,
-                                   stream);
+                                   stream, max_len);
 }
 
 }  // namespace
