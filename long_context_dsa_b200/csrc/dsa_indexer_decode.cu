@@ -343,7 +343,7 @@ bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Key-range splits per sequence: about `per_sm` units per SM (2 when every sequence has the
+// Key-range splits per sequence: about `per_sm` units per SM (4 when every sequence has the
 // same length; more when lengths differ, so that uneven units still balance), at least 8 key
 // tiles a unit.
 int dec_splits(int B, int nkt, int num_sms, int per_sm = 2) {
@@ -385,7 +385,7 @@ cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, in
     p.q_pos0 = q_pos0;
     p.n_kv = n_kv;
     p.topk = topk;
-    p.splits = dec_splits(B, nkt, num_sms, pc.seq_lens ? 6 : 2);
+    p.splits = dec_splits(B, nkt, num_sms, pc.seq_lens ? 6 : 4);
     p.tiles_per_split = (nkt + p.splits - 1) / p.splits;
     p.splits = (nkt + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty units
     p.hdr = static_cast<WsHeader*>(ws);
@@ -413,7 +413,7 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen) {
     const int nkt = (q_pos0 + 1 + 127) / 128;  // varlen: q_pos0 = the longest sequence - 1
-    int splits = dec_splits(B, nkt, num_sms, varlen ? 6 : 2);
+    int splits = dec_splits(B, nkt, num_sms, varlen ? 6 : 4);
     const int tps = (nkt + splits - 1) / splits;
     splits = (nkt + tps - 1) / tps;
     return static_cast<size_t>(B) * splits * topk * 8;
