@@ -353,35 +353,46 @@ __global__ void __launch_bounds__(WARPS * 32)
 }
 
 // Combine the split ranges of each (query row, KV head, query head):
-// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.
-template <bool OUT_BF16>
-__global__ void attn_merge_kernel(const float* __restrict__ part, int G, int D, int splits, int Hq, int Hkv,
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (ranges that saw no
+// key have m_s = -inf and drop out).  One block per unit, one warp per query head: lane s
+// holds range s's (m, l) (splits <= 32), the weights reach every lane by shuffles, and each
+// lane accumulates D/32 output columns with the ranges' loads independent of each other.
+template <int D, bool OUT_BF16>
+__global__ void attn_merge_kernel(const float* __restrict__ part, int G, int splits, int Hq, int Hkv,
                                   void* __restrict__ O) {
     const long long u = blockIdx.x;  // (row, g)
-    const int h = blockIdx.y;
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (h >= G) return;
     const long long row = u / Hkv;
     const int g = static_cast<int>(u % Hkv);
-    const float* p0 = part + (static_cast<size_t>(u) * splits * G + h) * (D + 2);
     const size_t sstride = static_cast<size_t>(G) * (D + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, p0[s * sstride + D]);
-    float L = 0.f;
-    for (int s = 0; s < splits; ++s) {
-        const float m = p0[s * sstride + D];
-        L += (m == -INFINITY) ? 0.f : exp2f(m - M) * p0[s * sstride + D + 1];
+    const float* p0 = part + (static_cast<size_t>(u) * splits * G + h) * (D + 2);
+    const float m = lane < splits ? __ldg(p0 + lane * sstride + D) : -INFINITY;
+    const float l = lane < splits ? __ldg(p0 + lane * sstride + D + 1) : 0.f;
+    float M = m;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    float L = f * l;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float acc[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int s2 = 0; s2 < splits; ++s2) {
+        const float fs = __shfl_sync(0xffffffffu, f, s2);
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) acc[i] += fs * __ldg(p0 + s2 * sstride + i * 32 + lane);
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            const float m = p0[s * sstride + D];
-            if (m != -INFINITY) acc += exp2f(m - M) * p0[s * sstride + d];
-        }
-        const size_t ob = (static_cast<size_t>(row) * Hq + g * G + h) * D + d;
+    const size_t ob = (static_cast<size_t>(row) * Hq + static_cast<size_t>(g) * G + h) * D;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
         if (OUT_BF16)
-            reinterpret_cast<__nv_bfloat16*>(O)[ob] = __float2bfloat16_rn(acc * inv);
+            reinterpret_cast<__nv_bfloat16*>(O)[ob + i * 32 + lane] = __float2bfloat16_rn(acc[i] * inv);
         else
-            reinterpret_cast<float*>(O)[ob] = acc * inv;
+            reinterpret_cast<float*>(O)[ob + i * 32 + lane] = acc[i] * inv;
     }
 }
 
@@ -442,11 +453,12 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
                                                                    scale_log2, O, splits, per, part, share, pg, hdr);
     if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
     const int G = Hq / Hkv;
-    dim3 mg(static_cast<unsigned>(units), static_cast<unsigned>(G));
+    // splits <= 32: attn_splits keeps at least 4 of the (at most 128) 16-key chunks in a range
+    if (splits > 32) return cudaErrorInvalidValue;
     if (out_bf16)
-        attn_merge_kernel<true><<<mg, 128, 0, stream>>>(part, G, D, splits, Hq, Hkv, O);
+        attn_merge_kernel<D, true><<<static_cast<unsigned>(units), G * 32, 0, stream>>>(part, G, splits, Hq, Hkv, O);
     else
-        attn_merge_kernel<false><<<mg, 128, 0, stream>>>(part, G, D, splits, Hq, Hkv, O);
+        attn_merge_kernel<D, false><<<static_cast<unsigned>(units), G * 32, 0, stream>>>(part, G, splits, Hq, Hkv, O);
     return cudaGetLastError();
 }
 
