@@ -178,8 +178,8 @@ def run_gpu(args, rank, world, local_rank):
 
     # ---- timed region: K steps of the shared-index group
     step_evs = [make_events() for _ in range(args.steps)]
-    clk = ClockSampler(local_rank, os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
-                                                else ".", f"clocks_rank{rank}.csv"))
+    import tempfile
+    clk = ClockSampler(local_rank, os.path.join(args.clocks_dir or tempfile.gettempdir(), f"clocks_rank{rank}.csv"))
     barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -832,6 +832,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=24)
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows for cpu_baseline (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--clocks-dir", default=None, help="keep the sampled clock log (clocks_rank<r>.csv) here")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench",
                     choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged"],
