@@ -122,3 +122,18 @@ def test_indexer_survivors_concentrated_in_one_lane_range():
     ora = oracle.indexer_scores(q[0], kk[0], w[0])
     frac = check_selection(idx, oracle.topk_select(ora, k), ora, 0, k, rtol=1e-3)
     assert frac > 0.9
+
+
+def test_decode_long_cache_uses_streaming_merge():
+    """A 1.7M-token cache: the position bitmap of the split merge would not fit in shared memory,
+    so the streaming merge of the partial lists runs; the selection is still the oracle's."""
+    B, L, H, d, k = 1, 1_700_000, 32, 128, 2048
+    g = synth.StructuredIndexer("long_decode", B, L, H, d, r=32, base_std=1.0, noise_std=0.2, seed=0)
+    kk = g.keys(0)
+    q, w = g.queries(0, L - 1, L)
+    ws = torch.zeros(dsa.idx_score_topk_workspace_size(B, 1, L - 1, L, H, d, k), dtype=torch.uint8, device=DEV)
+    idx = dsa.idx_score_topk(q.to(DEV), kk.to(DEV), w.to(DEV), k, q_pos0=L - 1, workspace=ws)
+    assert dsa.read_status(ws) == 0
+    ora = oracle.indexer_scores(q[0], kk[0], w[0], L - 1)
+    ora_idx = oracle.topk_select(ora, k, L - 1)
+    check_selection(idx.cpu().numpy()[0], ora_idx, ora, L - 1, k, rtol=1e-3)
