@@ -133,6 +133,33 @@ def adjacent_overlap(layers, dev, rows=2048):
             "mean": round(sum(fr) / len(fr), 4)}
 
 
+def pattern_search(layers, dev, rows=2048, n_f=2):
+    """The F/S search on this workload: every layer's own selection over the last `rows` query
+    rows (calibration rows), all pairwise overlaps, then the greedy pattern with n_f F layers."""
+    import time
+
+    import numpy as np
+    import torch
+    from long_context_dsa_b200 import dsa
+
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    p0 = L - rows
+    sel = [dsa.idx_score_topk(Lh["q_I"][:, p0:].contiguous(), Lh["k_I"], Lh["w"][:, p0:].contiguous(), TOPK,
+                              q_pos0=p0) for Lh in layers]
+    n = len(layers)
+    ov = np.zeros((n, n))
+    for f in range(n):
+        for j in range(f + 1, n):
+            ov[f, j] = float(dsa.idx_overlap(sel[f], sel[j]).double().mean().item()) / TOPK
+    pattern = dsa.layer_pattern_search(ov, n_f)
+    sec = time.perf_counter() - t0
+    return {"calibration_rows": f"last {rows} of {L}", "n_f": n_f, "pattern": pattern,
+            "mean_overlap_of_s_layers": round(float(np.mean([ov[max(i for i in range(j + 1) if pattern[i] == 'F'), j]
+                                                            for j in range(n) if pattern[j] == "S"])), 4),
+            "seconds": round(sec, 3)}
+
+
 def attn_traffic():
     """DRAM bytes of one full sparse-attention launch, scaled from the ncu capture of the tail case
     (4096 rows x 2048 selected keys: 2.492 GB read + 0.037 GB written) by selected (query, key) pairs;
@@ -212,6 +239,7 @@ def run_gpu(args, rank, world, local_rank):
     allf_idx = [allf_evs[3 * l].elapsed_time(allf_evs[3 * l + 1]) for l in range(N_LAYERS)]
     allf_step = allf_evs[0].elapsed_time(allf_evs[-1])
     overlap = adjacent_overlap(layers, dev)
+    search = pattern_search(layers, dev)
 
     # ---- end to end through the public API from pinned host memory
     e2e = None
@@ -260,6 +288,7 @@ def run_gpu(args, rank, world, local_rank):
                           "shared_indexer_ms": round(sum(idx_ms) / args.steps, 3),
                           "indexer_time_ratio": round(sum(allf_idx) / (sum(idx_ms) / args.steps), 3),
                           "adjacent_layer_overlap": overlap},
+        "pattern_search": search,
         "gpu_launches": launches,
         "clocks": clocks,
     }
