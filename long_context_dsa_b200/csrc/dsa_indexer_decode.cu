@@ -343,14 +343,21 @@ bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Key-range splits per sequence: about `per_sm` units per SM (4 when every sequence has the
+// Key-range splits per sequence: about `per_sm` units per SM (per_sm_for: 4 when every sequence has the
 // same length; more when lengths differ, so that uneven units still balance), at least 8 key
 // tiles a unit.
-int dec_splits(int B, int nkt, int num_sms, int per_sm = 2) {
+int dec_splits(int B, int nkt, int num_sms, int per_sm) {
     int s = (per_sm * num_sms + B - 1) / B;
     if (s > nkt / 8) s = nkt / 8;  // keep at least 8 key tiles per unit
     if (s < 1) s = 1;
     return s;
+}
+
+// Units per SM: more when lengths differ (uneven units balance better); for a few long
+// sequences the merge of their many partial lists would outweigh the finer split.
+int per_sm_for(int B, bool varlen) {
+    if (varlen) return 6;
+    return B >= 32 ? 4 : 2;
 }
 
 // Cache geometry of a decode launch.  Contiguous: k [B, n_kv, d], every sequence q_pos0 + 1 keys.
@@ -385,7 +392,7 @@ cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, in
     p.q_pos0 = q_pos0;
     p.n_kv = n_kv;
     p.topk = topk;
-    p.splits = dec_splits(B, nkt, num_sms, pc.seq_lens ? 6 : 4);
+    p.splits = dec_splits(B, nkt, num_sms, per_sm_for(B, pc.seq_lens != nullptr));
     p.tiles_per_split = (nkt + p.splits - 1) / p.splits;
     p.splits = (nkt + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty units
     p.hdr = static_cast<WsHeader*>(ws);
@@ -413,7 +420,7 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen) {
     const int nkt = (q_pos0 + 1 + 127) / 128;  // varlen: q_pos0 = the longest sequence - 1
-    int splits = dec_splits(B, nkt, num_sms, varlen ? 6 : 4);
+    int splits = dec_splits(B, nkt, num_sms, per_sm_for(B, varlen));
     const int tps = (nkt + splits - 1) / splits;
     splits = (nkt + tps - 1) / tps;
     return static_cast<size_t>(B) * splits * topk * 8;
