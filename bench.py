@@ -902,7 +902,7 @@ def main():
         out["cpu_baseline"] = {"value": round(v, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
                                "sample": sample}
     del layers
-    if not args.no_extra:
+    if not args.no_extra and world == 1:  # the extra measurements are single-GPU cases
         import torch
         torch.cuda.empty_cache()
         dev = torch.device("cuda", local_rank)
