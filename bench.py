@@ -325,19 +325,24 @@ def run_e2e(args, layers, shape, cache, ws, dev, stream, world=1):
         start = torch.cuda.Event()
         start.record(stream)
         s_in.wait_event(start)
-        landed = []
+        landed = []  # per layer: (indexer inputs in, attention inputs in)
         with torch.cuda.stream(s_in):
             for l, Lh in enumerate(layers):
-                for n, t in host_in[l].items():
-                    Lh[n].copy_(t, non_blocking=True)
-                e = torch.cuda.Event()
-                e.record(s_in)
-                landed.append(e)
+                evs = []
+                for group in (("q_I", "k_I", "w"), ("Q", "K", "V")):
+                    for n in group:
+                        if n in host_in[l]:
+                            Lh[n].copy_(host_in[l][n], non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(s_in)
+                    evs.append(e)
+                landed.append(evs)
         for l, Lh in enumerate(layers):
-            stream.wait_event(landed[l])
             if PATTERN[l] == "F":
+                stream.wait_event(landed[l][0])
                 dsa.idx_score_topk(Lh["q_I"], Lh["k_I"], Lh["w"], TOPK, out=cache.buf, workspace=ws, stream=stream)
                 cache.put(l, PATTERN)
+            stream.wait_event(landed[l][1])
             idx = dsa.idx_cache_get(cache, l, PATTERN)
             dsa.sparse_attn_topk(Lh["Q"], Lh["K"], Lh["V"], idx, o_dtype=torch.bfloat16, out=Lh["O"], workspace=ws,
                                  stream=stream)
