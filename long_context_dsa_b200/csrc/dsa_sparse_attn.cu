@@ -85,9 +85,6 @@ struct AttnCfg {
     }
 };
 
-// Chunks beyond the ring whose rows each warp prefetches into L2 (0: none).
-static constexpr int PREFETCH = 4;
-
 // Compile-time switches, so the plain path carries none of the bookkeeping of the others:
 // SPLIT: units cut into index ranges (few rows, e.g. decode); PAGED: K/V in a page pool;
 // SHARED: query rows share index rows.
@@ -203,17 +200,6 @@ __global__ void __launch_bounds__(WARPS * 32)
         for (int c = c0; c < c1; ++c) {
             issue(c + STAGES - 1, t_next);
             t_next = load_idx(c + STAGES);
-            if (PREFETCH) {
-                // rows of a chunk further ahead: pulled into L2 now, so the copies that fetch them
-                // later wait on L2 rather than on DRAM (more bytes in flight than the ring holds)
-                const int cp = c + STAGES + PREFETCH;
-                const int tp = cp < c1 ? load_idx(cp) : -1;
-                if (tp >= 0) {
-                    const size_t off = static_cast<size_t>(tp) * tok_stride;
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kb + off), "r"(D * 2) : "memory");
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vb + off), "r"(D * 2) : "memory");
-                }
-            }
             cp_async_wait<STAGES - 1>();
             __syncwarp();
             const int s = (SPLIT ? c - c0 : c) % STAGES;
