@@ -14,6 +14,9 @@ N > 1 runs under torchrun: every rank runs its own independent sequence
 time is the max over ranks and `value` counts the tokens of all ranks.
 Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on
 the host cores on a bounded sample of rows of the same workload.
+`--case cp` splits ONE sequence over the torchrun ranks instead
+(context-parallel prefill: zig-zag row blocks, an all-gather of the keys
+each step, strong scaling).
 """
 
 from __future__ import annotations
@@ -857,6 +860,75 @@ def run_ctx1m(args, dev):
             "full_prefill_estimate_tok_per_s": round(L1 / est_s, 1)}
 
 
+def run_cp(args, rank, world, local_rank):
+    """Context-parallel prefill of ONE 200K-token sequence split over the ranks (strong
+    scaling): every rank owns two zig-zag blocks of query rows, the keys (k_I of the F
+    layers, K and V of every layer) are all-gathered inside each step, then each rank runs
+    the layer group on its blocks as chunks of prefill.  With one rank the gather is the
+    local buffer itself and the step is the sequence in two chunks."""
+    import torch
+    from long_context_dsa_b200 import context_parallel as cp
+    from long_context_dsa_b200 import dsa, replicas
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    plan = cp.make_plan(L, world, rank)
+    full = make_layers(dev, rank=0, keep_indexer_all=False)   # the same sequence on every rank
+    layers, local_keys, gbufs = [], [], []
+    for Lh in full:
+        d = {n: cp.local_rows(Lh[n], plan) for n in ("q_I", "w", "Q") if n in Lh}
+        d["O"] = torch.empty((2, plan.blk, HQ, DH), dtype=torch.bfloat16, device=dev)
+        kl = {n: cp.local_rows(Lh[n], plan) for n in ("k_I", "K", "V") if n in Lh}
+        layers.append(d)
+        local_keys.append(kl)
+        gbufs.append({n: (torch.empty((2 * world, plan.blk) + tuple(t.shape[2:]), dtype=t.dtype, device=dev)
+                          if world > 1 else None) for n, t in kl.items()})
+    del full
+    torch.cuda.empty_cache()
+    gather_bytes = sum(t.numel() * t.element_size() for kl in local_keys for t in kl.values()) * (world - 1)
+    ws = torch.zeros(cp.workspace_size(plan, H_I, D_I, HQ, HKV, DH, DH, TOPK, o_dtype=dsa.DSA_BF16),
+                     dtype=torch.uint8, device=dev)
+    cache_buf = torch.empty((2, plan.blk, TOPK), dtype=torch.int32, device=dev)
+
+    def step():
+        for d, kl, gb in zip(layers, local_keys, gbufs):
+            for n, t in kl.items():
+                d[n] = cp.allgather_keys(t, plan, out=gb[n])
+        return cp.layer_group_forward(plan, layers, PATTERN, cache_buf, ws, H_I, D_I, HQ, HKV, DH, DH, TOPK,
+                                      o_dtype=dsa.DSA_BF16, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    replicas.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    launches = 0
+    for _ in range(args.steps):
+        n_idx, n_attn = step()
+        launches += n_idx + n_attn
+    t1.record(stream)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    dsa.check_status(ws)
+    ms = replicas.max_over_ranks(t0.elapsed_time(t1), dev) / args.steps
+    work = [cp.indexer_work(cp.make_plan(L, world, r)) for r in range(world)]
+    return {"metric": METRIC, "value": round(L / (ms / 1e3), 1), "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded structured generator; no dataset or trained weights)",
+            "config": {"workload": WORKLOAD + "; one sequence split over the ranks in zig-zag blocks",
+                       "seq_len": L, "global_batch": 1, "layers": N_LAYERS, "pattern": PATTERN, "topk": TOPK,
+                       "parallelism": f"context-parallel x{world}", "rows_per_block": plan.blk,
+                       "l2": "inputs larger than L2; no flush needed"},
+            "gpu_launches": launches,
+            "all_gather_bytes_per_rank_per_step": gather_bytes,
+            "indexer_work_max_over_mean": round(max(work) / (sum(work) / world), 5)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -869,9 +941,10 @@ def main():
     ap.add_argument("--clocks-dir", default=None, help="keep the sampled clock log (clocks_rank<r>.csv) here")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench",
-                    choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged"],
-                    help="profile: small single-kernel launches for ncu captures; decode / ctx1m: only that "
-                         "extra measurement, printed as one JSON line")
+                    choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged", "cp"],
+                    help="profile: small single-kernel launches for ncu captures; decode / ctx1m / ...: only "
+                         "that extra measurement, printed as one JSON line; cp: one 200K sequence split over "
+                         "the torchrun ranks (context-parallel prefill, strong scaling)")
     args = ap.parse_args()
     if args.case == "profile":
         run_profile_case(args)
@@ -901,6 +974,15 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
+    if args.case == "cp":
+        out = run_cp(args, rank, world, local_rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        return
     out, layers = run_gpu(args, rank, world, local_rank)
     if rank == 0 and args.cpu_rows > 0:
         v, total, sample, threads, meas = oracle_sample(layers, args.cpu_rows)
