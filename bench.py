@@ -782,15 +782,60 @@ def run_paged(args, dev):
     dsa.check_status(ws)
     ms = a.elapsed_time(b) / n
     kbytes = int(lens.sum()) * D_I * 2
-    del layers, k_pool
+    attn_ms = evs[1].elapsed_time(evs[2])
+    idx_ms = evs[0].elapsed_time(evs[1])
+
+    # the same step with the K/V cache stored as E4M3 codes + one scale per (token, KV head)
+    layers8 = []
+    for i in range(nl):
+        Q, Kp, Vp = layers[i]
+        layers[i] = None
+        K8, ks = synth.quantize_e4m3_rows(Kp)
+        del Kp
+        torch.cuda.empty_cache()
+        V8, vs = synth.quantize_e4m3_rows(Vp)
+        del Vp
+        torch.cuda.empty_cache()
+        layers8.append((Q, K8, ks, V8, vs))
+
+    def step8(evs=None):
+        if evs:
+            evs[0].record()
+        dsa.idx_score_topk_paged(q, k_pool, table, seq, w, TOPK, max_len, out=idx, workspace=ws)
+        if evs:
+            evs[1].record()
+        for (Q, K8, ks, V8, vs) in layers8:
+            dsa.sparse_attn_topk_paged_e4m3(Q, K8, ks, V8, vs, table, seq, idx, o_dtype=torch.bfloat16, out=O,
+                                            workspace=ws)
+        if evs:
+            evs[2].record()
+
+    for _ in range(3):
+        step8()
+    torch.cuda.synchronize()
+    a.record()
+    for i in range(n):
+        step8(evs if i == n - 1 else None)
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms8 = a.elapsed_time(b) / n
+    attn8_ms = evs[1].elapsed_time(evs[2])
+    gathered = B * TOPK * HKV * 2 * DH * nl           # K and V rows of every selected token (all lengths >= k)
+    del layers8, k_pool
     torch.cuda.empty_cache()
     return {"workload": f"paged decode: B={B} sequences of {int(lens.min())}-{int(lens.max())} tokens "
                         f"(mean {int(lens.mean())}) in shuffled {P}-token pages, 4 layers FSSS, "
                         f"H_I={H_I} d_I={D_I} top-{TOPK}, GQA {HQ}Q/{HKV}KV d={DH}",
             "tok_per_s": round(B / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
-            "indexer_ms": round(evs[0].elapsed_time(evs[1]), 4),
-            "attention_ms": round(evs[1].elapsed_time(evs[2]), 4),
-            "indexer_gbs": round(kbytes / (evs[0].elapsed_time(evs[1]) / 1e3) / 1e9, 1)}
+            "indexer_ms": round(idx_ms, 4),
+            "attention_ms": round(attn_ms, 4),
+            "attention_gathered_gbs": round(2 * gathered / (attn_ms / 1e3) / 1e9, 1),
+            "indexer_gbs": round(kbytes / (idx_ms / 1e3) / 1e9, 1),
+            "fp8_kv": {"tok_per_s": round(B / (ms8 / 1e3), 1), "ms_per_step": round(ms8, 4),
+                       "attention_ms": round(attn8_ms, 4),
+                       "attention_gathered_gbs": round(gathered / (attn8_ms / 1e3) / 1e9, 1),
+                       "cache": "E4M3 codes + fp32 scale per (token, KV head), quantized from the bf16 cache"}}
 
 
 def run_ctx1m(args, dev):

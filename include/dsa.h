@@ -249,6 +249,17 @@ DSA_API int sparse_attn_topk_shared(const void* Q, const void* K, const void* V,
  *   Hq/Hkv <= 8.  Indices >= seq_lens[b] or mapping to a page outside
  *   [0, num_pages) are skipped and flagged.  Workspace:
  *   sparse_attn_topk_workspace_size(B, 1, num_pages * page_size, ...).
+ *
+ * sparse_attn_topk_paged_e4m3: the same attention over a K/V cache kept
+ *   as OCP E4M3 codes (1 byte each, bias 7, max 448) with one fp32 scale
+ *   per (token, KV head): the real K row is code x k_scale, likewise V.
+ *   K8_pages, V8_pages [num_pages * page_size, Hkv, d] uint8 codes;
+ *   k_scale, v_scale [num_pages * page_size, Hkv] fp32; Q bf16 as above.
+ *   Arithmetic: Q is taken to fp16, K codes widen exactly to fp16 and the
+ *   K scale multiplies the fp32 score; V rows are code x scale rounded to
+ *   fp16; fp32 accumulation and softmax.  Same shapes, rules, flags and
+ *   workspace as sparse_attn_topk_paged.  The gather reads half the bytes
+ *   of a bf16 cache, which is what bounds decode attention.
  * ====================================================================== */
 DSA_API int idx_score_topk_paged_workspace_size(int B, int max_seq_len, int H_I, int d_I, int topk,
                                                 size_t* bytes);
@@ -261,6 +272,13 @@ DSA_API int sparse_attn_topk_paged(const void* Q, const void* K_pages, const voi
                                    int B, int page_size, int num_pages, int max_pages, int Hq, int Hkv,
                                    int d, int topk, float scale, void* O, int o_dtype,
                                    void* workspace, size_t workspace_bytes, void* stream);
+DSA_API int sparse_attn_topk_paged_e4m3(const void* Q, const void* K8_pages, const float* k_scale,
+                                        const void* V8_pages, const float* v_scale,
+                                        const int32_t* page_table, const int32_t* seq_lens,
+                                        const int32_t* idx, int B, int page_size, int num_pages,
+                                        int max_pages, int Hq, int Hkv, int d, int topk, float scale,
+                                        void* O, int o_dtype, void* workspace, size_t workspace_bytes,
+                                        void* stream);
 
 /* ======================================================================
  * F/S pattern search -- which layers of a group keep their indexer.

@@ -18,6 +18,10 @@ cudaError_t launch_topk_scores(const float* scores, int rows, int q_pos0, int n_
 cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, const int* idx, int B, int n_q,
                                int n_kv, int Hq, int Hkv, int d, int topk, float scale, void* O, bool out_bf16,
                                IdxShare share, KvPages pg, WsHeader* hdr, int num_sms, cudaStream_t stream);
+cudaError_t launch_sparse_attn_fp8_paged(const void* Q, const void* K8, const float* k_scale, const void* V8,
+                                         const float* v_scale, const int* idx, int B, int Hq, int Hkv, int d, int topk,
+                                         float scale, void* O, bool out_bf16, KvPages pg, WsHeader* hdr, int num_sms,
+                                         cudaStream_t stream);
 cudaError_t launch_indexer_decode_paged(const void* q, const void* k_pages, const int* page_table, const int* seq_lens,
                                         const float* w, int B, int max_len, int page_size, int num_pages,
                                         int max_pages, int H, int topk, int* idx_out, void* ws, int num_sms,
@@ -371,6 +375,40 @@ int sparse_attn_topk_paged(const void* Q, const void* K_pages, const void* V_pag
     const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages};
     return attn_common(Q, K_pages, V_pages, idx, B, 1, static_cast<int>(pool), Hq, Hkv, d, d, topk, scale, O,
                        o_dtype, dsa::kNoShare, workspace, workspace_bytes, stream, pages);
+}
+
+int sparse_attn_topk_paged_e4m3(const void* Q, const void* K8_pages, const float* k_scale, const void* V8_pages,
+                                const float* v_scale, const int32_t* page_table, const int32_t* seq_lens,
+                                const int32_t* idx, int B, int page_size, int num_pages, int max_pages, int Hq, int Hkv,
+                                int d, int topk, float scale, void* O, int o_dtype, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    if (!Q || !K8_pages || !k_scale || !V8_pages || !v_scale || !page_table || !seq_lens || !idx || !O)
+        return fail(DSA_ERR_INVALID_ARG, "NULL pointer");
+    if (page_size < 1 || num_pages < 1 || max_pages < 1)
+        return fail(DSA_ERR_INVALID_ARG, "bad page geometry page_size=%d num_pages=%d max_pages=%d", page_size,
+                    num_pages, max_pages);
+    const long long pool = static_cast<long long>(num_pages) * page_size;
+    if (pool > 0x7fffffffll) return fail(DSA_ERR_INVALID_ARG, "page pool too large");
+    int rc = check_attn_shape(V8_pages, B, 1, static_cast<int>(pool), Hq, Hkv, d, d, topk);
+    if (rc) return rc;
+    if (o_dtype != DSA_F32 && o_dtype != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "o_dtype must be F32 or BF16");
+    if (!aligned16(Q) || !aligned16(K8_pages) || !aligned16(V8_pages))
+        return fail(DSA_ERR_INVALID_ARG, "Q, K8_pages, V8_pages must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u)
+        return fail(DSA_ERR_INVALID_ARG, "scales must be 4-byte aligned");
+    size_t need;
+    if ((rc = sparse_attn_topk_workspace_size(B, 1, static_cast<int>(pool), Hq, Hkv, d, d, topk, &need))) return rc;
+    if ((rc = check_ws(workspace, workspace_bytes, need))) return rc;
+    if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(d));
+    int sms;
+    if ((rc = sm_count(&sms))) return rc;
+    const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages};
+    cudaError_t e = launch_sparse_attn_fp8_paged(Q, K8_pages, k_scale, V8_pages, v_scale, idx, B, Hq, Hkv, d, topk,
+                                                 scale, O, o_dtype == DSA_BF16, pages,
+                                                 static_cast<WsHeader*>(workspace), sms,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "sparse_attn_topk_paged_e4m3");
+    return DSA_OK;
 }
 
 int idx_score_topk_paged_workspace_size(int B, int max_seq_len, int H_I, int d_I, int topk, size_t* bytes) {

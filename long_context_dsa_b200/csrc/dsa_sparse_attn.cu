@@ -26,6 +26,9 @@
 //     (16-key chunks, 2 stages each) fit in shared memory at d = 128.  On
 //     B200 the number of warps in flight set the speed far more than the
 //     stages per warp did.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "dsa_common.cuh"
 
 namespace dsa {
@@ -462,6 +465,377 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------------
+// fp8 K/V cache (paged decode).  K and V are stored as OCP E4M3 codes with one fp32 scale per
+// (token, KV head): the real row is code x scale.  The gather moves half the bytes of bf16 rows.
+//   * Each warp's ring holds the codes (d bytes per row slice) of STAGES 16-key chunks, gathered
+//     with cp.async like the bf16 kernel; every row's two scales ride along with its index.
+//   * Before the MMAs the warp widens one chunk at a time into an fp16 scratch tile laid out
+//     like the bf16 ring (swizzled rows), so the same ldmatrix / mma.sync steps follow, in f16:
+//     K codes are widened exactly (every E4M3 value is an fp16 value) and the K scale multiplies
+//     the fp32 score; V codes are widened and multiplied by their row's scale in fp16, into the
+//     same scratch once the scores are done.  Q is taken to fp16 once per unit.
+//   * P is split into fp16 hi + lo parts, as the bf16 kernel does with bf16.
+// The split rule (and so the workspace) is the bf16 kernel's for the same d.
+template <int D, int STAGES, int WARPS>
+struct Fp8AttnCfg {
+    static constexpr int CHUNK = 16;
+    static constexpr int STAGE_BYTES = 2 * CHUNK * D;    // K codes, then V codes (d bytes a row)
+    static constexpr int RS = 2 * D;                     // fp16 scratch row stride (bytes)
+    static constexpr int SCRATCH = CHUNK * RS;
+    static constexpr int META = STAGES * CHUNK * 12;     // per stage and key: pool row, K scale, V scale
+    static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + SCRATCH + META;
+    static constexpr size_t SMEM = static_cast<size_t>(WARPS) * WARP_BYTES;
+    static constexpr int SEG8 = D / 16;                  // 16-byte segments of a code row slice
+    static constexpr int KEYS_PER_INSN = 32 / SEG8;
+    static_assert(32 % SEG8 == 0 && (CHUNK * SEG8) % 32 == 0, "row slices split evenly over the warp");
+    __device__ static __forceinline__ uint32_t at(int r, int sg) {
+        return static_cast<uint32_t>(r * RS + ((sg ^ (r & 7)) << 4));
+    }
+};
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+// two E4M3 codes (low byte first) -> two fp16 values, exactly
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// Widen one chunk's code rows (16 rows of D bytes at `src`) into the fp16 scratch tile; with
+// SCALED, row r is multiplied by scale[r].
+template <class C, bool SCALED>
+__device__ __forceinline__ void widen_chunk(const unsigned char* src, uint32_t scr_s, const float* scale, int lane) {
+#pragma unroll
+    for (int i = 0; i < C::CHUNK * C::SEG8 / 32; ++i) {
+        const int q = i * 32 + lane;
+        const int r = q / C::SEG8, sg = q % C::SEG8;
+        const uint4 v = *reinterpret_cast<const uint4*>(src + q * 16);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            h[2 * j] = e4m3x2_to_f16x2(w[j]);
+            h[2 * j + 1] = e4m3x2_to_f16x2(w[j] >> 16);
+        }
+        if (SCALED) {
+            const __half2 sc = __float2half2_rn(scale[r]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                __half2 x = *reinterpret_cast<__half2*>(&h[j]);
+                x = __hmul2(x, sc);
+                h[j] = *reinterpret_cast<uint32_t*>(&x);
+            }
+        }
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(scr_s + C::at(r, 2 * sg)), "r"(h[0]), "r"(h[1]),
+                     "r"(h[2]), "r"(h[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(scr_s + C::at(r, 2 * sg + 1)), "r"(h[4]),
+                     "r"(h[5]), "r"(h[6]), "r"(h[7])
+                     : "memory");
+    }
+}
+
+template <int D, int STAGES, int WARPS, bool OUT_BF16, bool SPLIT>
+__global__ void __launch_bounds__(WARPS * 32, 1)
+    sparse_attn_fp8_kernel(const __nv_bfloat16* __restrict__ Q, const unsigned char* __restrict__ K8,
+                           const float* __restrict__ k_scale, const unsigned char* __restrict__ V8,
+                           const float* __restrict__ v_scale, const int* __restrict__ idx, int B, int Hq, int Hkv,
+                           int topk, float scale_log2, void* __restrict__ O, int splits, int chunks_per_split,
+                           float* __restrict__ part, KvPages pg, WsHeader* hdr) {
+    using C = Fp8AttnCfg<D, STAGES, WARPS>;
+    constexpr int CHUNK = C::CHUNK;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char* ring = smem + warp * C::WARP_BYTES;
+    const uint32_t ring_s = smem_u32(ring);
+    const uint32_t scr_s = ring_s + STAGES * C::STAGE_BYTES;
+    int* srow = reinterpret_cast<int*>(ring + STAGES * C::STAGE_BYTES + C::SCRATCH);
+    float* sks = reinterpret_cast<float*>(srow + STAGES * CHUNK);
+    float* svs = sks + STAGES * CHUNK;
+
+    const int G = Hq / Hkv;
+    const long long units = static_cast<long long>(B) * Hkv;  // one query per sequence
+    const long long items = SPLIT ? units * splits : units;
+    const int nchunks = (topk + CHUNK - 1) / CHUNK;
+    const size_t tok_stride = static_cast<size_t>(Hkv) * D;  // bytes per token row of the code pools
+
+    const int qn = lane >> 2;
+    const int hc = 2 * (lane & 3);
+    const int lrow = lane & 7, lq = lane >> 3;
+    const int k_key_off = ((lq & 1) ? 8 : 0) + lrow, k_d_off = (lq >= 2) ? 8 : 0;
+    const int v_key_off = ((lq >= 2) ? 8 : 0) + lrow, v_d_off = (lq & 1) ? 8 : 0;
+    const int seg = lane % C::SEG8, sub = lane / C::SEG8;
+
+    for (long long it = static_cast<long long>(blockIdx.x) * WARPS + warp; it < items;
+         it += static_cast<long long>(gridDim.x) * WARPS) {
+        const long long u = SPLIT ? it / splits : it;
+        const int sp = SPLIT ? static_cast<int>(it % splits) : 0;
+        const int c0 = SPLIT ? sp * chunks_per_split : 0;
+        const int c1 = SPLIT ? min(nchunks, c0 + chunks_per_split) : nchunks;
+        const long long b = u / Hkv;
+        const int g = static_cast<int>(u % Hkv);
+        const int* irow = idx + b * topk;
+        const unsigned char* kb = K8 + static_cast<size_t>(g) * D;
+        const unsigned char* vb = V8 + static_cast<size_t>(g) * D;
+        const int n_valid = min(__ldg(pg.lens + b), pg.max_pages * pg.page_size);
+
+        // The index of key `lane` of chunk c is read two chunks ahead of its gather and mapped to
+        // its pool row (page-table read, checks) one chunk ahead, so neither dependent read sits
+        // on the critical path; the row's two scales travel with its codes (cp.async).
+        auto load_raw = [&](int c) -> int {
+            const int kk = c * CHUNK + lane;
+            return (lane < CHUNK && kk < topk) ? __ldg(irow + kk) : -1;
+        };
+        auto map_row = [&](int t) -> int {  // logical position -> pool row (-1: padding or flagged)
+            if (t < -1 || t >= n_valid) {
+                raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
+                t = -1;
+            }
+            if (t >= 0) {
+                const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + t / pg.page_size);
+                if (page < 0 || page >= pg.num_pages) {
+                    raise_status(hdr, DSA_STATUS_BAD_INDEX, page);
+                    t = -1;
+                } else {
+                    t = page * pg.page_size + t % pg.page_size;
+                }
+            }
+            return t;
+        };
+        auto issue = [&](int c, int tsel) {
+            if (c < c1) {
+                const int s = (SPLIT ? c - c0 : c) % STAGES;
+                if (lane < CHUNK) {
+                    srow[s * CHUNK + lane] = tsel;
+                    const size_t so = static_cast<size_t>(tsel >= 0 ? tsel : 0) * Hkv + g;
+                    const uint32_t nb = tsel >= 0 ? 4u : 0u;
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(sks + s * CHUNK + lane)),
+                                 "l"(k_scale + so), "r"(nb)
+                                 : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(svs + s * CHUNK + lane)),
+                                 "l"(v_scale + so), "r"(nb)
+                                 : "memory");
+                }
+                const uint32_t kst = ring_s + s * C::STAGE_BYTES;
+                const uint32_t vst = kst + CHUNK * D;
+#pragma unroll
+                for (int i = 0; i < CHUNK / C::KEYS_PER_INSN; ++i) {
+                    const int key = i * C::KEYS_PER_INSN + sub;
+                    const int t = __shfl_sync(0xffffffffu, tsel, key);
+                    const uint32_t nb = t >= 0 ? 16u : 0u;
+                    const size_t off = static_cast<size_t>(t >= 0 ? t : 0) * tok_stride + seg * 16;
+                    cp_async16(kst + key * D + seg * 16, kb + off, nb);
+                    cp_async16(vst + key * D + seg * 16, vb + off, nb);
+                }
+            }
+            cp_async_commit();
+        };
+
+        // Q^T fragments in fp16
+        uint32_t qf[D / 16][2];
+        {
+            const bool live = qn < G;
+            const __nv_bfloat16* qp = Q + (static_cast<size_t>(b) * Hq + g * G + (live ? qn : 0)) * D + hc;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t raw = live ? __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 * e)) : 0u;
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
+                    qf[ks][e] = pack_f16(f.x, f.y);
+                }
+            }
+        }
+        float o[D / 16][4];
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
+
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < STAGES - 1; ++c) issue(c0 + c, map_row(load_raw(c0 + c)));
+        int t_next = map_row(load_raw(c0 + STAGES - 1));  // pool rows of the next chunk to gather
+        int r_next = load_raw(c0 + STAGES);                // raw indices of the one after
+
+        for (int c = c0; c < c1; ++c) {
+            issue(c + STAGES - 1, t_next);
+            t_next = map_row(r_next);
+            r_next = load_raw(c + STAGES + 1);
+            cp_async_wait<STAGES - 1>();
+            __syncwarp();
+            const int s = (SPLIT ? c - c0 : c) % STAGES;
+            const unsigned char* kcodes = ring + s * C::STAGE_BYTES;
+            const int* si = srow + s * CHUNK;
+            const float* ks_ = sks + s * CHUNK;
+            const float* vs_ = svs + s * CHUNK;
+            // ---- K codes -> fp16 scratch, S^T = K Q^T (two accumulation chains)
+            widen_chunk<C, false>(kcodes, scr_s, nullptr, lane);
+            __syncwarp();
+            float sacc[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(scr_s + C::at(k_key_off, 2 * ks + k_d_off / 8), a0, a1, a2, a3);
+                if (ks & 1)
+                    mma_f16(s2, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                else
+                    mma_f16(sacc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+            }
+            __syncwarp();  // every lane has its K fragments before V overwrites the scratch
+            // ---- V codes x their row scales -> fp16 scratch (read after the softmax)
+            widen_chunk<C, true>(kcodes + CHUNK * D, scr_s, vs_, lane);
+            // ---- mask, K scale, softmax scale, online softmax
+            const bool v0 = si[qn] >= 0, v1 = si[qn + 8] >= 0;
+            const float f0 = ks_[qn] * scale_log2, f1 = ks_[qn + 8] * scale_log2;
+            float mx[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                sacc[j] = v0 ? (sacc[j] + s2[j]) * f0 : -INFINITY;
+                sacc[2 + j] = v1 ? (sacc[2 + j] + s2[2 + j]) * f1 : -INFINITY;
+                mx[j] = fmaxf(sacc[j], sacc[2 + j]);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
+            }
+            float alpha[2], mnew[2], p[4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                mnew[j] = fmaxf(mrun[j], mx[j]);
+                alpha[j] = (mnew[j] == -INFINITY) ? 1.f : exp2f(mrun[j] - mnew[j]);
+                mrun[j] = mnew[j];
+                lrun[j] *= alpha[j];
+                p[j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[j] - mnew[j]);
+                p[2 + j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[2 + j] - mnew[j]);
+                lrun[j] += p[j] + p[2 + j];
+            }
+            const uint32_t h01 = pack_f16(p[0], p[1]);
+            const uint32_t h23 = pack_f16(p[2], p[3]);
+            const float2 r01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+            const float2 r23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+            const uint32_t phi0 = movm_t(h01), phi1 = movm_t(h23);
+            const uint32_t plo0 = movm_t(pack_f16(p[0] - r01.x, p[1] - r01.y));
+            const uint32_t plo1 = movm_t(pack_f16(p[2] - r23.x, p[3] - r23.y));
+            __syncwarp();  // the V scratch is complete
+            // ---- O^T = alpha * O^T + V^T P
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+                o[dt][0] *= alpha[0];
+                o[dt][1] *= alpha[1];
+                o[dt][2] *= alpha[0];
+                o[dt][3] *= alpha[1];
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(scr_s + C::at(v_key_off, 2 * dt + v_d_off / 8), a0, a1, a2, a3);
+                mma_f16(o[dt], a0, a1, a2, a3, phi0, phi1);
+                mma_f16(o[dt], a0, a1, a2, a3, plo0, plo1);
+            }
+            __syncwarp();  // stage s and the scratch are free
+        }
+        cp_async_wait<0>();
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) lrun[j] += __shfl_xor_sync(0xffffffffu, lrun[j], off);
+        }
+        if (SPLIT) {
+            float* pb = part + static_cast<size_t>(it) * G * (D + 2);
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+                const int d0 = dt * 16 + qn;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = hc + j;
+                    if (h < G) {
+                        pb[h * (D + 2) + d0] = o[dt][j];
+                        pb[h * (D + 2) + d0 + 8] = o[dt][2 + j];
+                    }
+                }
+            }
+            if (qn == 0) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = hc + j;
+                    if (h < G) {
+                        pb[h * (D + 2) + D] = mrun[j];
+                        pb[h * (D + 2) + D + 1] = lrun[j];
+                    }
+                }
+            }
+            continue;
+        }
+        const float inv0 = lrun[0] > 0.f ? 1.f / lrun[0] : 0.f;
+        const float inv1 = lrun[1] > 0.f ? 1.f / lrun[1] : 0.f;
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt) {
+            const int d0 = dt * 16 + qn;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = hc + j;
+                if (h < G) {
+                    const float inv = j ? inv1 : inv0;
+                    const size_t ob = (static_cast<size_t>(b) * Hq + g * G + h) * D;
+                    if (OUT_BF16) {
+                        __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(O) + ob;
+                        op[d0] = __float2bfloat16_rn(o[dt][j] * inv);
+                        op[d0 + 8] = __float2bfloat16_rn(o[dt][2 + j] * inv);
+                    } else {
+                        float* op = reinterpret_cast<float*>(O) + ob;
+                        op[d0] = o[dt][j] * inv;
+                        op[d0 + 8] = o[dt][2 + j] * inv;
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int D, int STAGES, int WARPS, int SPLIT_WARPS>
+static cudaError_t launch_attn_fp8_t(const __nv_bfloat16* Q, const unsigned char* K8, const float* k_scale,
+                                     const unsigned char* V8, const float* v_scale, const int* idx, int B, int Hq,
+                                     int Hkv, int topk, float scale, void* O, bool out_bf16, KvPages pg, WsHeader* hdr,
+                                     int num_sms, cudaStream_t stream) {
+    using C = Fp8AttnCfg<D, STAGES, WARPS>;
+    const long long units = static_cast<long long>(B) * Hkv;
+    const int nchunks = (topk + C::CHUNK - 1) / C::CHUNK;
+    int per = nchunks;
+    // the bf16 kernel's split rule for this d, so sparse_attn_part_bytes sizes the workspace
+    const int splits = attn_splits(units, nchunks, SPLIT_WARPS, num_sms, &per);
+    using KernFn = void (*)(const __nv_bfloat16*, const unsigned char*, const float*, const unsigned char*,
+                            const float*, const int*, int, int, int, int, float, void*, int, int, float*, KvPages,
+                            WsHeader*);
+    static const KernFn table[2][2] = {
+        {sparse_attn_fp8_kernel<D, STAGES, WARPS, false, false>, sparse_attn_fp8_kernel<D, STAGES, WARPS, false, true>},
+        {sparse_attn_fp8_kernel<D, STAGES, WARPS, true, false>, sparse_attn_fp8_kernel<D, STAGES, WARPS, true, true>}};
+    KernFn kern = table[out_bf16 ? 1 : 0][splits > 1 ? 1 : 0];
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
+    if (e != cudaSuccess) return e;
+    long long grid = num_sms;
+    const long long need = (units * splits + WARPS - 1) / WARPS;
+    if (grid > need) grid = need;
+    if (grid < 1) grid = 1;
+    float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(hdr) + kWsHeaderBytes);
+    kern<<<static_cast<int>(grid), WARPS * 32, C::SMEM, stream>>>(Q, K8, k_scale, V8, v_scale, idx, B, Hq, Hkv, topk,
+                                                                   scale * 1.4426950408889634f, O, splits, per, part,
+                                                                   pg, hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    const int G = Hq / Hkv;
+    if (splits > 32) return cudaErrorInvalidValue;
+    if (out_bf16)
+        attn_merge_kernel<D, true><<<static_cast<unsigned>(units), G * 32, 0, stream>>>(part, G, splits, Hq, Hkv, O);
+    else
+        attn_merge_kernel<D, false><<<static_cast<unsigned>(units), G * 32, 0, stream>>>(part, G, splits, Hq, Hkv, O);
+    return cudaGetLastError();
+}
+
 // Bytes of split-range state the sparse attention needs beyond the status word.
 size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms) {
     if (d != 128 && d != 64) return 0;
@@ -488,6 +862,25 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
     if (d == 64)
         return launch_attn_t<64, 16, 2, kAttnWarpsD64, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
                                                         out_bf16, share, pg, hdr, num_sms, stream);
+    return cudaErrorNotSupported;
+}
+
+// fp8 (E4M3 + per-row scale) paged K/V: one query per sequence.
+cudaError_t launch_sparse_attn_fp8_paged(const void* Q, const void* K8, const float* k_scale, const void* V8,
+                                         const float* v_scale, const int* idx, int B, int Hq, int Hkv, int d, int topk,
+                                         float scale, void* O, bool out_bf16, KvPages pg, WsHeader* hdr, int num_sms,
+                                         cudaStream_t stream) {
+    auto q = static_cast<const __nv_bfloat16*>(Q);
+    auto k = static_cast<const unsigned char*>(K8);
+    auto v = static_cast<const unsigned char*>(V8);
+    // 4 stages of 4 KB codes + a 4 KB fp16 scratch per warp: 10 warps per SM at d = 128 (measured
+    // on B200 against 3 stages x 12 or 13 warps)
+    if (d == 128)
+        return launch_attn_fp8_t<128, 4, 10, kAttnWarpsD128>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale,
+                                                              O, out_bf16, pg, hdr, num_sms, stream);
+    if (d == 64)
+        return launch_attn_fp8_t<64, 3, 16, kAttnWarpsD64>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale, O,
+                                                            out_bf16, pg, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }
 

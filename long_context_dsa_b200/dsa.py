@@ -30,6 +30,7 @@ ABI_SYMBOLS = (
     "layer_group_forward_workspace_size", "layer_group_forward",
     "idx_score_topk_noalloc", "idx_overlap", "layer_pattern_search",
     "idx_score_topk_paged_workspace_size", "idx_score_topk_paged", "sparse_attn_topk_paged",
+    "sparse_attn_topk_paged_e4m3",
 )
 
 
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
         "idx_score_topk_paged_workspace_size": ([i, i, i, i, i, psz], i),
         "idx_score_topk_paged": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp, sz, vp], i),
         "sparse_attn_topk_paged": ([vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, i, vp, sz, vp], i),
+        "sparse_attn_topk_paged_e4m3": ([vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, i, vp, sz,
+                                         vp], i),
         "layer_pattern_search": ([ctypes.POINTER(ctypes.c_double), i, i, ctypes.c_char_p], i),
     }
     for name, (args, res) in sig.items():
@@ -375,6 +378,38 @@ def sparse_attn_topk_paged(Q, K_pages, V_pages, page_table, seq_lens, idx, scale
                                         _ptr(idx), B, page_size, num_pages, max_pages, Hq, Hkv, d, topk,
                                         float(scale or 0.0), _ptr(out), od, _ptr(workspace), workspace.numel(),
                                         _stream(stream)))
+    return out
+
+
+def sparse_attn_topk_paged_e4m3(Q, K8_pages, k_scale, V8_pages, v_scale, page_table, seq_lens, idx,
+                                scale: float | None = None, o_dtype=torch.float32, out=None, workspace=None,
+                                stream=None) -> torch.Tensor:
+    """sparse_attn_topk_paged over an fp8 cache: K8_pages, V8_pages [num_pages, page_size, Hkv, d]
+    E4M3 codes (uint8), k_scale, v_scale [num_pages, page_size, Hkv] fp32 (real row = code x scale)."""
+    _need(Q, torch.bfloat16, "Q")
+    for t, n in ((K8_pages, "K8_pages"), (V8_pages, "V8_pages")):
+        _need(t, torch.uint8, n)
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, torch.float32, n)
+    _need(page_table, torch.int32, "page_table")
+    _need(seq_lens, torch.int32, "seq_lens")
+    _need(idx, torch.int32, "idx")
+    B, Hq, d = Q.shape
+    num_pages, page_size, Hkv = K8_pages.shape[0], K8_pages.shape[1], K8_pages.shape[2]
+    if tuple(k_scale.shape) != (num_pages, page_size, Hkv) or tuple(v_scale.shape) != (num_pages, page_size, Hkv):
+        raise ValueError("scales must be [num_pages, page_size, Hkv]")
+    max_pages = page_table.shape[1]
+    topk = idx.shape[-1]
+    od = DSA_F32 if o_dtype == torch.float32 else DSA_BF16
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=o_dtype, device=Q.device)
+    if workspace is None:
+        workspace = _workspace(sparse_attn_topk_workspace_size(B, 1, num_pages * page_size, Hq, Hkv, d, d, topk),
+                               Q.device)
+    _check(lib().sparse_attn_topk_paged_e4m3(_ptr(Q), _ptr(K8_pages), _ptr(k_scale), _ptr(V8_pages), _ptr(v_scale),
+                                             _ptr(page_table), _ptr(seq_lens), _ptr(idx), B, page_size, num_pages,
+                                             max_pages, Hq, Hkv, d, topk, float(scale or 0.0), _ptr(out), od,
+                                             _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 
 

@@ -14,6 +14,7 @@ method's arithmetic.
 
 from .dsa_oracle import (  # noqa: F401
     e4m3_decode,
+    dequantize_e4m3,
     indexer_scores,
     indexer_scores_fp8,
     topk_select,

@@ -66,6 +66,14 @@ def e4m3_decode(codes) -> np.ndarray:
     return v
 
 
+def dequantize_e4m3(codes, scale) -> np.ndarray:
+    """Real values of per-row scaled E4M3 codes: codes [..., d] (uint8), scale [...]
+    (one factor per row); value = e4m3_decode(code) * scale, in float64.  This is the
+    fp8 storage the indexer's k_I and q_I use and the fp8 K/V cache: a code times its
+    row's scale."""
+    return e4m3_decode(codes) * _f64(scale)[..., None]
+
+
 # ---------------------------------------------------------------------------
 # a1: indexer scores
 # ---------------------------------------------------------------------------

@@ -182,6 +182,41 @@ def test_fp8_power_of_two_rescale_changes_only_scale():
     assert np.array_equal(a[:, others], b[:, others])
 
 
+def test_dequantize_e4m3_code_points_and_scales():
+    """Code x its row's scale, from the format: 0x38 = 1, 0x7E = 448, 0xB8 = -1, 0x01 = 2^-9."""
+    codes = np.array([[0x38, 0x7E], [0xB8, 0x01]], np.uint8)
+    v = oracle.dequantize_e4m3(codes, np.array([0.5, 3.0], np.float32))
+    assert v.tolist() == [[0.5, 224.0], [-3.0, 3 * 2.0 ** -9]]
+    # unit scales reduce to the plain decode; the scale of one row touches that row only
+    c = np.arange(256, dtype=np.uint8).reshape(16, 16)
+    ones = oracle.dequantize_e4m3(c, np.ones(16))
+    assert np.array_equal(ones, e4m3_decode(c), equal_nan=True)
+    sc = np.ones(16)
+    sc[5] = 0.25
+    v2 = oracle.dequantize_e4m3(c, sc)
+    assert np.array_equal(v2[5], e4m3_decode(c[5]) * 0.25, equal_nan=True)
+    assert np.array_equal(np.delete(v2, 5, 0), np.delete(ones, 5, 0), equal_nan=True)
+
+
+def test_fp8_kv_cache_scales_act_on_scores_and_values():
+    """Attention over a dequantized fp8 cache: a power-of-two K scale on every row equals that
+    factor on Q; a V scale on every row scales the output by it."""
+    rng = np.random.default_rng(5)
+    Q = rng.standard_normal((1, 4, 16))
+    K8 = synth.quantize_e4m3_rows(synth.normal((40, 2, 16), 21))[0].numpy()
+    V8 = synth.quantize_e4m3_rows(synth.normal((40, 2, 16), 22))[0].numpy()
+    ks = np.full((40, 2), 0.01)
+    vs = np.full((40, 2), 0.02)
+    idx = np.array([[0, 3, 17, 39, -1]])
+    base = sparse_attention(Q, oracle.dequantize_e4m3(K8, ks), oracle.dequantize_e4m3(V8, vs), idx)
+    k4 = sparse_attention(Q, oracle.dequantize_e4m3(K8, 4 * ks), oracle.dequantize_e4m3(V8, vs), idx)
+    q4 = sparse_attention(4 * Q, oracle.dequantize_e4m3(K8, ks), oracle.dequantize_e4m3(V8, vs), idx)
+    v3 = sparse_attention(Q, oracle.dequantize_e4m3(K8, ks), oracle.dequantize_e4m3(V8, 3 * vs), idx)
+    np.testing.assert_allclose(k4, q4, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(v3, 3 * base, rtol=1e-13, atol=0)
+    assert not np.allclose(k4, base)
+
+
 # --------------------------------------------------------------------------
 # top-k
 # --------------------------------------------------------------------------
