@@ -521,6 +521,52 @@ def run_profile_case(args):
                       "indexer_queries": nq_i, "attn_queries": nq_a, "n_kv": L}))
 
 
+def run_profile_paged(args):
+    """Small paged decode case for ncu captures of the gather attention: 64 sequences of 12500
+    tokens in shuffled 64-token pages (K/V pools 0.8 GB each in bf16, larger than L2), random
+    top-2048 selections, GQA 32/4, d=128.  Each iteration launches the bf16-cache kernel, then
+    the fp8-cache kernel on the same cache quantized to E4M3 + per-row scales."""
+    import numpy as np
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    dev = torch.device("cuda", 0)
+    B, P, Lseq = 64, 64, 12500
+    rng = np.random.default_rng(4000)
+    lens = np.full(B, Lseq, np.int32)
+    max_pages = (Lseq + P - 1) // P
+    num_pages = B * max_pages
+    table = torch.from_numpy(rng.permutation(num_pages).astype(np.int32).reshape(B, max_pages)).to(dev)
+    seq = torch.from_numpy(lens).to(dev)
+    idx = torch.from_numpy(np.stack([np.sort(rng.choice(Lseq, size=TOPK, replace=False))
+                                     for _ in range(B)]).astype(np.int32)).to(dev)
+    Kp = synth.normal((num_pages, P, HKV, DH), synth.seed_for(4000, "profpaged", "K"), dev, dtype=torch.bfloat16)
+    Vp = synth.normal((num_pages, P, HKV, DH), synth.seed_for(4000, "profpaged", "V"), dev, dtype=torch.bfloat16)
+    Q = synth.normal((B, HQ, DH), synth.seed_for(4000, "profpaged", "Q"), dev, dtype=torch.bfloat16)
+    K8, ks = synth.quantize_e4m3_rows(Kp)
+    V8, vs = synth.quantize_e4m3_rows(Vp)
+    ws = torch.zeros(dsa.sparse_attn_topk_workspace_size(B, 1, num_pages * P, HQ, HKV, DH, DH, TOPK),
+                     dtype=torch.uint8, device=dev)
+    O = torch.empty((B, HQ, DH), dtype=torch.bfloat16, device=dev)
+    t_b, t_8 = [], []
+    for it in range(args.warmup + args.steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        dsa.sparse_attn_topk_paged(Q, Kp, Vp, table, seq, idx, o_dtype=torch.bfloat16, out=O, workspace=ws)
+        e[1].record()
+        dsa.sparse_attn_topk_paged_e4m3(Q, K8, ks, V8, vs, table, seq, idx, o_dtype=torch.bfloat16, out=O,
+                                        workspace=ws)
+        e[2].record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            t_b.append(e[0].elapsed_time(e[1]))
+            t_8.append(e[1].elapsed_time(e[2]))
+    dsa.check_status(ws)
+    by = B * TOPK * HKV * DH * 2          # K and V codes gathered (bf16: twice this)
+    print(json.dumps({"case": "profile_paged", "bf16_ms": min(t_b), "bf16_gathered_gbs": 2 * by / min(t_b) / 1e6,
+                      "fp8_ms": min(t_8), "fp8_gathered_gbs": by / min(t_8) / 1e6}))
+
+
 def run_decode(args, dev):
     """Decode step: 64 sequences, one new token each, at a 200000-token cache; 4 layers FSSS
     (H_I=32, d_I=128, top-2048; attention 32 query / 4 KV heads, d=128)."""
@@ -986,13 +1032,17 @@ def main():
     ap.add_argument("--clocks-dir", default=None, help="keep the sampled clock log (clocks_rank<r>.csv) here")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench",
-                    choices=["bench", "profile", "decode", "decode_mha", "ctx1m", "mtp", "paged", "cp"],
+                    choices=["bench", "profile", "profile_paged", "decode", "decode_mha", "ctx1m", "mtp", "paged",
+                             "cp"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m / ...: only "
                          "that extra measurement, printed as one JSON line; cp: one 200K sequence split over "
                          "the torchrun ranks (context-parallel prefill, strong scaling)")
     args = ap.parse_args()
     if args.case == "profile":
         run_profile_case(args)
+        return
+    if args.case == "profile_paged":
+        run_profile_paged(args)
         return
     if args.case in ("decode", "decode_mha", "ctx1m", "mtp", "paged"):
         import torch

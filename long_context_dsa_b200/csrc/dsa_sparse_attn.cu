@@ -516,11 +516,15 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
 // SCALED, row r is multiplied by scale[r].
 template <class C, bool SCALED>
 __device__ __forceinline__ void widen_chunk(const unsigned char* src, uint32_t scr_s, const float* scale, int lane) {
+    constexpr int N = C::CHUNK * C::SEG8 / 32;  // 16-byte pieces per lane
+    uint4 in[N];                                // all loads first: the stores below are ordered asm
 #pragma unroll
-    for (int i = 0; i < C::CHUNK * C::SEG8 / 32; ++i) {
+    for (int i = 0; i < N; ++i) in[i] = *reinterpret_cast<const uint4*>(src + (i * 32 + lane) * 16);
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
         const int q = i * 32 + lane;
         const int r = q / C::SEG8, sg = q % C::SEG8;
-        const uint4 v = *reinterpret_cast<const uint4*>(src + q * 16);
+        const uint4 v = in[i];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t h[8];
 #pragma unroll
