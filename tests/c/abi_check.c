@@ -48,6 +48,14 @@ int main(void) {
                                4096, NULL) == DSA_ERR_INVALID_ARG); /* table holds 640 < 1000 tokens */
     CHECK(sparse_attn_topk_paged(p, p, p, NULL, fake, fake, 2, 64, 10, 10, 32, 4, 128, 64, 0.f, p, DSA_F32, p,
                                  4096, NULL) == DSA_ERR_INVALID_ARG); /* no page table */
+    const float* fs = (const float*)p;
+    CHECK(sparse_attn_topk_paged_e4m3(p, p, NULL, p, fs, fake, fake, fake, 2, 64, 10, 10, 32, 4, 128, 64, 0.f, p,
+                                      DSA_F32, p, 4096, NULL) == DSA_ERR_INVALID_ARG); /* no K scales */
+    CHECK(sparse_attn_topk_paged_e4m3(p, p, fs, p, fs, fake, fake, fake, 2, 64, 10, 10, 32, 4, 96, 64, 0.f, p,
+                                      DSA_F32, p, 4096, NULL) == DSA_ERR_UNSUPPORTED); /* d = 96 */
+    CHECK(sparse_attn_topk_paged_e4m3(p, p, (const float*)(size_t)0x1002, p, fs, fake, fake, fake, 2, 64, 10, 10,
+                                      32, 4, 128, 64, 0.f, p, DSA_F32, p, 4096, NULL)
+          == DSA_ERR_INVALID_ARG); /* misaligned scales */
     CHECK(idx_overlap(fake, NULL, 4, 8, fake, NULL) == DSA_ERR_INVALID_ARG);
     CHECK(idx_overlap(fake, fake, 0, 8, fake, NULL) == DSA_ERR_INVALID_ARG);
     size_t n = 0;
