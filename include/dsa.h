@@ -52,7 +52,7 @@ extern "C" {
 /* ---- status codes ---------------------------------------------------- */
 #define DSA_OK               0
 #define DSA_ERR_INVALID_ARG  1  /* bad shape, null pointer, bad pattern, small workspace */
-#define DSA_ERR_UNSUPPORTED  2  /* valid request this build has no kernel for            */
+#define DSA_ERR_UNSUPPORTED  2  /* valid request the library has no kernel for           */
 #define DSA_ERR_CUDA         3  /* a CUDA runtime call or launch failed                  */
 #define DSA_ERR_TIMEOUT      4  /* a bounded device-side wait gave up (status word)      */
 #define DSA_ERR_DEVICE       5  /* a kernel rejected its data (status word), e.g. an
@@ -69,7 +69,7 @@ extern "C" {
 #define DSA_STATUS_NAN_SCORE  0x4   /* top-k met a NaN score                    */
 #define DSA_STATUS_OVERFLOW   0x8   /* a candidate buffer would have overflowed */
 
-/* Largest top-k this build selects. */
+/* Largest top-k the library selects. */
 #define DSA_TOPK_MAX 2048
 
 /* Thread-local text of the last error raised on this host thread. */
