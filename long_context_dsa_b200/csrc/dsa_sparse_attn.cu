@@ -469,28 +469,33 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
 // fp8 K/V cache (paged decode).  K and V are stored as OCP E4M3 codes with one fp32 scale per
 // (token, KV head): the real row is code x scale.  The gather moves half the bytes of bf16 rows.
 //   * Each warp's ring holds the codes (d bytes per row slice) of STAGES 16-key chunks, gathered
-//     with cp.async like the bf16 kernel; every row's two scales ride along with its index.
-//   * Before the MMAs the warp widens one chunk at a time into an fp16 scratch tile laid out
-//     like the bf16 ring (swizzled rows), so the same ldmatrix / mma.sync steps follow, in f16:
-//     K codes are widened exactly (every E4M3 value is an fp16 value) and the K scale multiplies
-//     the fp32 score; V codes are widened and multiplied by their row's scale in fp16, into the
-//     same scratch once the scores are done.  Q is taken to fp16 once per unit.
-//   * P is split into fp16 hi + lo parts, as the bf16 kernel does with bf16.
+//     with cp.async like the bf16 kernel (16-byte segments XOR-swizzled by row); every row's two
+//     scales ride along.  Indices are read two chunks ahead, pool rows one chunk ahead.
+//   * The MMA fragments come straight from the codes (f16 MMAs; every E4M3 value is an fp16
+//     value):  S^T = K Q^T takes each lane's 4 consecutive code bytes of a key row as its A
+//     elements, which permutes d inside each 16-wide k-step; Q's fragments are loaded with the
+//     same permutation, so the dot products are unchanged.  O^T += V^T P loads the V codes with
+//     ldmatrix.trans (pairs of bytes as 16-bit elements), regroups the bytes so each register
+//     holds two keys of one d, and widens them; rows of O^T (d) come out interleaved (even d,
+//     then odd d, per 16) and are written back in place.
+//   * The K scale multiplies the fp32 score; V is widened times its key's scale in fp16 (one
+//     rounding of code x fp16(scale)); P is split into fp16 hi + lo parts.
 // The split rule (and so the workspace) is the bf16 kernel's for the same d.
 template <int D, int STAGES, int WARPS>
 struct Fp8AttnCfg {
     static constexpr int CHUNK = 16;
     static constexpr int STAGE_BYTES = 2 * CHUNK * D;    // K codes, then V codes (d bytes a row)
-    static constexpr int RS = 2 * D;                     // fp16 scratch row stride (bytes)
-    static constexpr int SCRATCH = CHUNK * RS;
     static constexpr int META = STAGES * CHUNK * 12;     // per stage and key: pool row, K scale, V scale
-    static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + SCRATCH + META;
+    static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + META;
     static constexpr size_t SMEM = static_cast<size_t>(WARPS) * WARP_BYTES;
     static constexpr int SEG8 = D / 16;                  // 16-byte segments of a code row slice
     static constexpr int KEYS_PER_INSN = 32 / SEG8;
-    static_assert(32 % SEG8 == 0 && (CHUNK * SEG8) % 32 == 0, "row slices split evenly over the warp");
+    static_assert(D == 64 || D == 128, "code rows of 4 or 8 segments");
+    // byte offset of segment sg of code row r: the 8 rows one ldmatrix (or one quarter of the
+    // warp's 4-byte loads) touches land in 8 different 16-byte bank groups
     __device__ static __forceinline__ uint32_t at(int r, int sg) {
-        return static_cast<uint32_t>(r * RS + ((sg ^ (r & 7)) << 4));
+        const int f = D == 128 ? (r & 7) : ((r >> 1) & 3);
+        return static_cast<uint32_t>(r * D + ((sg ^ f) << 4));
     }
 };
 
@@ -511,43 +516,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
     const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
-
-// Widen one chunk's code rows (16 rows of D bytes at `src`) into the fp16 scratch tile; with
-// SCALED, row r is multiplied by scale[r].
-template <class C, bool SCALED>
-__device__ __forceinline__ void widen_chunk(const unsigned char* src, uint32_t scr_s, const float* scale, int lane) {
-    constexpr int N = C::CHUNK * C::SEG8 / 32;  // 16-byte pieces per lane
-    uint4 in[N];                                // all loads first: the stores below are ordered asm
-#pragma unroll
-    for (int i = 0; i < N; ++i) in[i] = *reinterpret_cast<const uint4*>(src + (i * 32 + lane) * 16);
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-        const int q = i * 32 + lane;
-        const int r = q / C::SEG8, sg = q % C::SEG8;
-        const uint4 v = in[i];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t h[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            h[2 * j] = e4m3x2_to_f16x2(w[j]);
-            h[2 * j + 1] = e4m3x2_to_f16x2(w[j] >> 16);
-        }
-        if (SCALED) {
-            const __half2 sc = __float2half2_rn(scale[r]);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                __half2 x = *reinterpret_cast<__half2*>(&h[j]);
-                x = __hmul2(x, sc);
-                h[j] = *reinterpret_cast<uint32_t*>(&x);
-            }
-        }
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(scr_s + C::at(r, 2 * sg)), "r"(h[0]), "r"(h[1]),
-                     "r"(h[2]), "r"(h[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(scr_s + C::at(r, 2 * sg + 1)), "r"(h[4]),
-                     "r"(h[5]), "r"(h[6]), "r"(h[7])
-                     : "memory");
-    }
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t x, __half2 s) {
+    __half2 v = __hmul2(*reinterpret_cast<__half2*>(&x), s);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
 }
 
 template <int D, int STAGES, int WARPS, bool OUT_BF16, bool SPLIT>
@@ -563,8 +539,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char* ring = smem + warp * C::WARP_BYTES;
     const uint32_t ring_s = smem_u32(ring);
-    const uint32_t scr_s = ring_s + STAGES * C::STAGE_BYTES;
-    int* srow = reinterpret_cast<int*>(ring + STAGES * C::STAGE_BYTES + C::SCRATCH);
+    int* srow = reinterpret_cast<int*>(ring + STAGES * C::STAGE_BYTES);
     float* sks = reinterpret_cast<float*>(srow + STAGES * CHUNK);
     float* svs = sks + STAGES * CHUNK;
 
@@ -574,12 +549,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     const int nchunks = (topk + CHUNK - 1) / CHUNK;
     const size_t tok_stride = static_cast<size_t>(Hkv) * D;  // bytes per token row of the code pools
 
-    const int qn = lane >> 2;
-    const int hc = 2 * (lane & 3);
-    const int lrow = lane & 7, lq = lane >> 3;
-    const int k_key_off = ((lq & 1) ? 8 : 0) + lrow, k_d_off = (lq >= 2) ? 8 : 0;
-    const int v_key_off = ((lq >= 2) ? 8 : 0) + lrow, v_d_off = (lq & 1) ? 8 : 0;
+    const int qn = lane >> 2;           // key row (S^T) / head column (Q, P) / d pair (V^T) of this lane
+    const int c4 = lane & 3;
+    const int hc = 2 * c4;              // first of the two head columns this lane owns in C tiles
     const int seg = lane % C::SEG8, sub = lane / C::SEG8;
+    // ldmatrix.x4.trans over V: matrices (keys 0-7 | keys 8-15) x (segment dt | dt + 1)
+    const int v_key = ((lane >> 3) & 1) * 8 + (lane & 7), v_seg = lane >> 4;
 
     for (long long it = static_cast<long long>(blockIdx.x) * WARPS + warp; it < items;
          it += static_cast<long long>(gridDim.x) * WARPS) {
@@ -639,26 +614,26 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     const int t = __shfl_sync(0xffffffffu, tsel, key);
                     const uint32_t nb = t >= 0 ? 16u : 0u;
                     const size_t off = static_cast<size_t>(t >= 0 ? t : 0) * tok_stride + seg * 16;
-                    cp_async16(kst + key * D + seg * 16, kb + off, nb);
-                    cp_async16(vst + key * D + seg * 16, vb + off, nb);
+                    cp_async16(kst + C::at(key, seg), kb + off, nb);
+                    cp_async16(vst + C::at(key, seg), vb + off, nb);
                 }
             }
             cp_async_commit();
         };
 
-        // Q^T fragments in fp16
+        // Q^T fragments in fp16, d permuted like the K fragments: k-step ks takes d = 16 ks + 4 c4
+        // + {0,1} (rows 2 c4, 2 c4 + 1 of B) and + {2,3} (rows 2 c4 + 8, 2 c4 + 9)
         uint32_t qf[D / 16][2];
         {
             const bool live = qn < G;
-            const __nv_bfloat16* qp = Q + (static_cast<size_t>(b) * Hq + g * G + (live ? qn : 0)) * D + hc;
+            const __nv_bfloat16* qp = Q + (static_cast<size_t>(b) * Hq + g * G + (live ? qn : 0)) * D + 4 * c4;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const uint32_t raw = live ? __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 * e)) : 0u;
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
-                    qf[ks][e] = pack_f16(f.x, f.y);
-                }
+                const uint2 raw = live ? __ldg(reinterpret_cast<const uint2*>(qp + ks * 16)) : make_uint2(0u, 0u);
+                const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+                const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+                qf[ks][0] = pack_f16(f0.x, f0.y);
+                qf[ks][1] = pack_f16(f1.x, f1.y);
             }
         }
         float o[D / 16][4];
@@ -679,26 +654,24 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             cp_async_wait<STAGES - 1>();
             __syncwarp();
             const int s = (SPLIT ? c - c0 : c) % STAGES;
-            const unsigned char* kcodes = ring + s * C::STAGE_BYTES;
+            const uint32_t kst = ring_s + s * C::STAGE_BYTES;
+            const uint32_t vst = kst + CHUNK * D;
             const int* si = srow + s * CHUNK;
             const float* ks_ = sks + s * CHUNK;
             const float* vs_ = svs + s * CHUNK;
-            // ---- K codes -> fp16 scratch, S^T = K Q^T (two accumulation chains)
-            widen_chunk<C, false>(kcodes, scr_s, nullptr, lane);
-            __syncwarp();
+            // ---- S^T = K Q^T: A rows qn and qn + 8 take code bytes 16 ks + 4 c4 .. + 3
             float sacc[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(scr_s + C::at(k_key_off, 2 * ks + k_d_off / 8), a0, a1, a2, a3);
+                const uint32_t w0 = lds32(kst + C::at(qn, ks) + 4 * c4);
+                const uint32_t w1 = lds32(kst + C::at(qn + 8, ks) + 4 * c4);
+                const uint32_t a0 = e4m3x2_to_f16x2(w0), a2 = e4m3x2_to_f16x2(w0 >> 16);
+                const uint32_t a1 = e4m3x2_to_f16x2(w1), a3 = e4m3x2_to_f16x2(w1 >> 16);
                 if (ks & 1)
                     mma_f16(s2, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
                 else
                     mma_f16(sacc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
             }
-            __syncwarp();  // every lane has its K fragments before V overwrites the scratch
-            // ---- V codes x their row scales -> fp16 scratch (read after the softmax)
-            widen_chunk<C, true>(kcodes + CHUNK * D, scr_s, vs_, lane);
             // ---- mask, K scale, softmax scale, online softmax
             const bool v0 = si[qn] >= 0, v1 = si[qn + 8] >= 0;
             const float f0 = ks_[qn] * scale_log2, f1 = ks_[qn + 8] * scale_log2;
@@ -729,20 +702,33 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             const uint32_t phi0 = movm_t(h01), phi1 = movm_t(h23);
             const uint32_t plo0 = movm_t(pack_f16(p[0] - r01.x, p[1] - r01.y));
             const uint32_t plo1 = movm_t(pack_f16(p[2] - r23.x, p[3] - r23.y));
-            __syncwarp();  // the V scratch is complete
-            // ---- O^T = alpha * O^T + V^T P
+            // V scales of the keys this lane's A elements hold: 2 c4, 2 c4 + 1 and 8 + 2 c4, 9 + 2 c4
+            const __half2 vs_lo = __floats2half2_rn(vs_[2 * c4], vs_[2 * c4 + 1]);
+            const __half2 vs_hi = __floats2half2_rn(vs_[8 + 2 * c4], vs_[9 + 2 * c4]);
+            // ---- O^T = alpha * O^T + V^T P, two 16-d blocks per ldmatrix.x4.trans
 #pragma unroll
-            for (int dt = 0; dt < D / 16; ++dt) {
-                o[dt][0] *= alpha[0];
-                o[dt][1] *= alpha[1];
-                o[dt][2] *= alpha[0];
-                o[dt][3] *= alpha[1];
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(scr_s + C::at(v_key_off, 2 * dt + v_d_off / 8), a0, a1, a2, a3);
-                mma_f16(o[dt], a0, a1, a2, a3, phi0, phi1);
-                mma_f16(o[dt], a0, a1, a2, a3, plo0, plo1);
+            for (int dt = 0; dt < D / 16; dt += 2) {
+                uint32_t r[4];
+                ldsm_x4_t(vst + C::at(v_key, dt + v_seg), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    // r[2e]: keys 0-7, r[2e+1]: keys 8-15; bytes (k0,d) (k0,d+1) (k1,d) (k1,d+1)
+                    const uint32_t lo = __byte_perm(r[2 * e], 0u, 0x3120);
+                    const uint32_t hi = __byte_perm(r[2 * e + 1], 0u, 0x3120);
+                    const uint32_t a0 = hmul2_u32(e4m3x2_to_f16x2(lo), vs_lo);        // d even
+                    const uint32_t a1 = hmul2_u32(e4m3x2_to_f16x2(lo >> 16), vs_lo);  // d odd
+                    const uint32_t a2 = hmul2_u32(e4m3x2_to_f16x2(hi), vs_hi);
+                    const uint32_t a3 = hmul2_u32(e4m3x2_to_f16x2(hi >> 16), vs_hi);
+                    float(&od)[4] = o[dt + e];
+                    od[0] *= alpha[0];
+                    od[1] *= alpha[1];
+                    od[2] *= alpha[0];
+                    od[3] *= alpha[1];
+                    mma_f16(od, a0, a1, a2, a3, phi0, phi1);
+                    mma_f16(od, a0, a1, a2, a3, plo0, plo1);
+                }
             }
-            __syncwarp();  // stage s and the scratch are free
+            __syncwarp();  // stage s is free
         }
         cp_async_wait<0>();
 #pragma unroll
@@ -750,18 +736,16 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) lrun[j] += __shfl_xor_sync(0xffffffffu, lrun[j], off);
         }
+        // O^T rows of block dt: row qn holds d = 16 dt + 2 qn, row qn + 8 holds d = 16 dt + 2 qn + 1
         if (SPLIT) {
             float* pb = part + static_cast<size_t>(it) * G * (D + 2);
 #pragma unroll
             for (int dt = 0; dt < D / 16; ++dt) {
-                const int d0 = dt * 16 + qn;
+                const int d0 = dt * 16 + 2 * qn;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int h = hc + j;
-                    if (h < G) {
-                        pb[h * (D + 2) + d0] = o[dt][j];
-                        pb[h * (D + 2) + d0 + 8] = o[dt][2 + j];
-                    }
+                    if (h < G) *reinterpret_cast<float2*>(pb + h * (D + 2) + d0) = make_float2(o[dt][j], o[dt][2 + j]);
                 }
             }
             if (qn == 0) {
@@ -780,7 +764,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         const float inv1 = lrun[1] > 0.f ? 1.f / lrun[1] : 0.f;
 #pragma unroll
         for (int dt = 0; dt < D / 16; ++dt) {
-            const int d0 = dt * 16 + qn;
+            const int d0 = dt * 16 + 2 * qn;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int h = hc + j;
@@ -789,12 +773,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     const size_t ob = (static_cast<size_t>(b) * Hq + g * G + h) * D;
                     if (OUT_BF16) {
                         __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(O) + ob;
-                        op[d0] = __float2bfloat16_rn(o[dt][j] * inv);
-                        op[d0 + 8] = __float2bfloat16_rn(o[dt][2 + j] * inv);
+                        *reinterpret_cast<__nv_bfloat162*>(op + d0) =
+                            __floats2bfloat162_rn(o[dt][j] * inv, o[dt][2 + j] * inv);
                     } else {
                         float* op = reinterpret_cast<float*>(O) + ob;
-                        op[d0] = o[dt][j] * inv;
-                        op[d0 + 8] = o[dt][2 + j] * inv;
+                        *reinterpret_cast<float2*>(op + d0) = make_float2(o[dt][j] * inv, o[dt][2 + j] * inv);
                     }
                 }
             }
@@ -877,13 +860,12 @@ cudaError_t launch_sparse_attn_fp8_paged(const void* Q, const void* K8, const fl
     auto q = static_cast<const __nv_bfloat16*>(Q);
     auto k = static_cast<const unsigned char*>(K8);
     auto v = static_cast<const unsigned char*>(V8);
-    // 4 stages of 4 KB codes + a 4 KB fp16 scratch per warp: 10 warps per SM at d = 128 (measured
-    // on B200 against 3 stages x 12 or 13 warps)
+    // 3 stages of 4 KB codes per warp: 16 warps per SM at d = 128
     if (d == 128)
-        return launch_attn_fp8_t<128, 4, 10, kAttnWarpsD128>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale,
+        return launch_attn_fp8_t<128, 3, 16, kAttnWarpsD128>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale,
                                                               O, out_bf16, pg, hdr, num_sms, stream);
     if (d == 64)
-        return launch_attn_fp8_t<64, 3, 16, kAttnWarpsD64>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale, O,
+        return launch_attn_fp8_t<64, 4, 16, kAttnWarpsD64>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale, O,
                                                             out_bf16, pg, hdr, num_sms, stream);
     return cudaErrorNotSupported;
 }
