@@ -128,6 +128,10 @@ def _rank_main(rank, world, port, out):
                     full = Lh[name].float()
                     got = cp.allgather_keys(cp.local_rows(full, plan), plan)
                     ok_gather &= bool(torch.equal(got[:, : s["L"]], full)) and bool(torch.all(got[:, s["L"]:] == 0))
+                    # into a caller buffer, as the bench does every step (stale contents overwritten)
+                    buf = torch.full((2 * world, plan.blk) + tuple(full.shape[2:]), 7.0)
+                    got2 = cp.allgather_keys(cp.local_rows(full, plan), plan, out=buf)
+                    ok_gather &= got2.data_ptr() == buf.data_ptr() and bool(torch.equal(got2, got))
                     g[name] = got
             res.append(g)
         # each block is a chunk of prefill over the gathered keys (oracle arithmetic)
