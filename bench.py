@@ -441,12 +441,37 @@ def oracle_sample(layers, n_rows: int, seed: int = 0):
     per_idx = t_idx / work_idx
     per_att = t_att / work_att
     total = per_idx * n_f * (L * (L + 1) / 2) + per_att * N_LAYERS * gathered_rows(L, TOPK)
-    threads = torch.get_num_threads()
+    threads = cpu_info()["cores"]
     sample = (f"{len(rows)} query rows (seeded, spread over t, last row included) through the {PATTERN} group: "
               f"indexer+top-k on {n_f} F layers and attention on {N_LAYERS} layers; "
               f"{t_idx + t_att:.1f} s measured, extrapolated by algorithmic work "
               f"(sum of t+1 for the indexer, sum of min(k,t+1) for attention)")
     return L / total, total, sample, threads, t_idx + t_att
+
+
+def cpu_info():
+    """Host cores this process may run on, the CPU model and numpy's BLAS thread count (the
+    oracle's matrix products run in numpy's BLAS; everything else is single-threaded numpy)."""
+    cores = len(os.sched_getaffinity(0))
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    blas = None
+    try:
+        import numpy  # noqa: F401  (loads the BLAS library threadpoolctl inspects)
+        import threadpoolctl
+        info = [p for p in threadpoolctl.threadpool_info() if p.get("user_api") == "blas"]
+        if info:
+            blas = {"library": info[0].get("internal_api"), "threads": info[0].get("num_threads")}
+    except Exception:
+        pass
+    return {"cores": cores, "cpu_model": model, "blas": blas}
 
 
 def run_reference(args, rank, world):
@@ -467,7 +492,7 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD, "seq_len": L, "pattern": PATTERN},
             "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host": cpu_info()},
             "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -1082,7 +1107,7 @@ def main():
     if rank == 0 and args.cpu_rows > 0:
         v, total, sample, threads, meas = oracle_sample(layers, args.cpu_rows)
         out["cpu_baseline"] = {"value": round(v, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
-                               "sample": sample}
+                               "sample": sample, "host": cpu_info()}
     del layers
     if not args.no_extra and world == 1:  # the extra measurements are single-GPU cases
         import torch

@@ -69,6 +69,15 @@ extern "C" {
 #define DSA_STATUS_NAN_SCORE  0x4   /* top-k met a NaN score                    */
 #define DSA_STATUS_OVERFLOW   0x8   /* a candidate buffer would have overflowed */
 
+/* Test hook of the timeout path.  The 32-bit word at byte offset 8 of a
+ * workspace (inside its status word) must be zero in normal use (a zeroed
+ * workspace and dsa_reset_status() leave it so).  If it holds this value,
+ * the TMA producers of idx_score_topk's kernels withhold the first key tile
+ * of each CTA: every bounded wait on that tile runs out (about 2 s), the
+ * kernel winds down without faulting and dsa_check_status() returns
+ * DSA_ERR_TIMEOUT.  The indices written by such a call are meaningless. */
+#define DSA_TEST_WITHHOLD_TILE 0x5D5A7E57
+
 /* Largest top-k the library selects. */
 #define DSA_TOPK_MAX 2048
 
@@ -133,8 +142,12 @@ DSA_API int idx_scores(const void* q_I, const float* q_scale, const void* k_I, c
 /* ======================================================================
  * idx_topk_scores -- the top-k selection alone, on a given score array.
  *
- * Same selection code and rule as idx_score_topk; used to check the
- * selection bit-exactly against a reference on identical scores.
+ * The same selection rule as idx_score_topk, from the same building blocks
+ * (per-warp candidate buffers, radix select, merge of sorted sub-buffers);
+ * it prunes with the exact radix select only, while the fused kernel first
+ * prunes to a superset by a score histogram.  Given identical scores both
+ * give identical indices; used to check a selection bit-exactly against a
+ * reference on a score array.
  *   scores  [rows, ld] fp32 (row i uses columns 0 .. q_pos0+i; ld >= n_kv)
  *   idx_out [rows, topk] int32, layout as above.
  * Scores in the causal range must not be NaN (DSA_STATUS_NAN_SCORE).

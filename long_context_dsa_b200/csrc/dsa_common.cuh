@@ -18,9 +18,17 @@ namespace dsa {
 struct WsHeader {
     int status;        // DSA_STATUS_* bits, OR-ed by kernels
     int detail;        // first offending value (bad index) or wait site
-    int pad[62];
+    int test_hook;     // DSA_TEST_WITHHOLD_TILE: the TMA producers withhold their first key tile
+    int pad[61];
 };
 static constexpr size_t kWsHeaderBytes = 256;
+
+// True when the host asked the TMA-fed kernels to withhold their first key tile, so that
+// every bounded wait on it runs out and the kernel reports DSA_STATUS_TIMEOUT (the test of
+// the timeout path; no fault, no unbounded wait).
+__device__ __forceinline__ bool test_withhold_tile(const WsHeader* h) {
+    return h && *reinterpret_cast<const volatile int*>(&h->test_hook) == DSA_TEST_WITHHOLD_TILE;
+}
 
 __device__ __forceinline__ void raise_status(WsHeader* h, int bits, int detail) {
     if (h) {

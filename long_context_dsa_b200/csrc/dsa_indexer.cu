@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(320, 1)
             uint32_t it = 0, wt = 0;
             bool ok = true;
             int pend_q = -1;
+            const bool withhold = test_withhold_tile(p.hdr);  // timeout test: first key tile never sent
             for (int r = 0; ok; ++r) {
                 const int ti = tile_index(blockIdx.x, r, G);
                 if (ti >= p.n_tiles) break;
@@ -165,6 +166,7 @@ __global__ void __launch_bounds__(320, 1)
                     const int s = it % C::STAGES;
                     const uint32_t rr = it / C::STAGES;
                     if (rr > 0 && !mbar_wait(&kv_empty[s], (rr - 1) & 1)) { ok = false; break; }
+                    if (withhold && it == 0) continue;  // nothing issued: the waits on this stage run out
                     mbar_arrive_expect_tx(&kv_full[s], C::A_STAGE);
                     for (int kb = 0; kb < C::KB; ++kb)
                         tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128, &tmap_k, kb * C::BOX_X,

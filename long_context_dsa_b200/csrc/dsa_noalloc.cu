@@ -102,7 +102,19 @@ extern "C" DSA_API int idx_score_topk_noalloc(const void* q_I, const float* q_sc
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return set_err(DSA_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(e));
     const size_t fit = room / per_cta;
-    const int max_ctas = static_cast<int>(fit < static_cast<size_t>(sms) ? fit : static_cast<size_t>(sms));
+    int max_ctas = static_cast<int>(fit < static_cast<size_t>(sms) ? fit : static_cast<size_t>(sms));
+    // The estimate above is exact for the prefill kernel, whose scratch grows with its grid.  The
+    // one-query decode kernel sizes its partial lists by a split count that is a step function of
+    // the SM count it is given, so check the bytes the launch will really use and shrink the grid
+    // until they fit.
+    while (max_ctas > 1 &&
+           dsa::indexer_workspace_bytes(B, n_q, q_pos0, n_kv, H_I, d_I, topk, dtype, max_ctas) > room)
+        --max_ctas;
+    if (dsa::indexer_workspace_bytes(B, n_q, q_pos0, n_kv, H_I, d_I, topk, dtype, max_ctas) > room) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "the problem needs more than the %zu scratch bytes of the no-alloc array", room);
+        return set_err(DSA_ERR_UNSUPPORTED, msg);
+    }
     void* scratch = nullptr;
     if ((rc = scratch_address(&scratch))) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -1,8 +1,8 @@
 // dsa_topk_scores.cu -- the per-row top-k alone, on a given fp32 score array.
 //
-// Same selection code (dsa_topk.cuh) and rule as the fused indexer; exists
-// so the selection can be checked bit for bit against a reference that
-// scores rows independently.  One 128-thread CTA owns a row at a time;
+// The same selection rule and building blocks (dsa_topk.cuh) as the fused
+// indexer, pruning with the exact radix select only; exists so a selection
+// can be checked bit for bit against a reference on a given score array.  One 128-thread CTA owns a row at a time;
 // the candidate buffer lives in the CTA's shared memory.
 #include "dsa_topk.cuh"
 

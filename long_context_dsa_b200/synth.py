@@ -149,3 +149,48 @@ def quantize_e4m3_rows(x: torch.Tensor):
     y = (xf / scale.unsqueeze(-1)).clamp_(-448.0, 448.0)
     codes = y.to(torch.float8_e4m3fn).view(torch.uint8)
     return codes.contiguous(), scale.contiguous()
+
+
+def integer_indexer(name: str, B: int, L: int, H: int, d: int, lo: int, hi: int, seed: int = 0,
+                    w_steps: int = 4, q_rows: int | None = None):
+    """Indexer inputs whose scores are exact in fp32 whatever the summation order:
+    q_I [B, L, H, d] and k_I [B, L, d] hold integers drawn uniformly from lo..hi (exact in
+    bf16), w [B, L, H] holds multiples of 1/w_steps in [0, 1].  With |lo|, |hi| <= 8 and
+    d <= 128 every dot product is an integer of magnitude <= 8192 and every partial sum over
+    heads a multiple of 1/w_steps well inside fp32's 24-bit significand, so any two correct
+    implementations produce identical scores and, with ties to the lower index, identical
+    selections.  Small ranges give many equal scores (ties) and many zero scores (ReLU).
+    ``q_rows``: draw only that many query rows (q_I and w of the last q_rows positions; a
+    decode step needs one row against a long key cache)."""
+    nq = L if q_rows is None else q_rows
+
+    def ints(shape, tag):
+        g = _gen(seed_for(seed, name, tag), "cpu")
+        return torch.randint(lo, hi + 1, shape, generator=g, dtype=torch.int32)
+
+    q = ints((B, nq, H, d), "q").to(torch.bfloat16)
+    k = ints((B, L, d), "k").to(torch.bfloat16)
+    g = _gen(seed_for(seed, name, "w"), "cpu")
+    w = torch.randint(0, w_steps + 1, (B, nq, H), generator=g, dtype=torch.int32).to(torch.float32) / w_steps
+    return q.contiguous(), k.contiguous(), w.contiguous()
+
+
+def integer_indexer_e4m3(name: str, B: int, L: int, H: int, d: int, lo: int, hi: int, seed: int = 0,
+                         q_rows: int | None = None):
+    """fp8 counterpart of ``integer_indexer``: E4M3 codes of integers lo..hi (every integer of
+    magnitude <= 16 is an E4M3 value), per-row scales that are powers of two (2^-3 .. 2^1), and
+    w in multiples of 1/4.  Returns (q8 uint8 [B,L,H,d], q_scale fp32 [B,L,H], k8 uint8 [B,L,d],
+    k_scale fp32 [B,L], w fp32 [B,L,H]); scores of the real values code x scale stay exact in
+    fp32.  ``q_rows`` as for ``integer_indexer``."""
+    nq = L if q_rows is None else q_rows
+
+    def ints(shape, tag, a, b):
+        g = _gen(seed_for(seed, name, tag), "cpu")
+        return torch.randint(a, b + 1, shape, generator=g, dtype=torch.int32)
+
+    q8 = ints((B, nq, H, d), "q8", lo, hi).to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+    k8 = ints((B, L, d), "k8", lo, hi).to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+    q_scale = torch.exp2(ints((B, nq, H), "q_scale", -3, 1).to(torch.float32))
+    k_scale = torch.exp2(ints((B, L), "k_scale", -3, 1).to(torch.float32))
+    w = ints((B, nq, H), "w", 0, 4).to(torch.float32) / 4
+    return q8.contiguous(), q_scale.contiguous(), k8.contiguous(), k_scale.contiguous(), w.contiguous()

@@ -550,3 +550,31 @@ def test_structured_generator_overlap_in_reported_band():
         idx.append(topk_select(sc, k, q_pos0=L // 2))
     ov = topk_overlap(idx[0], idx[1], k, q_pos0=L // 2)
     assert 0.70 <= ov <= 1.0, ov
+
+
+def test_integer_generator_scores_are_exact_integers_over_four():
+    """The exact-selection GPU tests rely on integer q/k and quarter-step w giving scores
+    that fp32 holds exactly: check the oracle's rounded fp32 scores against int64 arithmetic
+    (4 * score = sum_h (4 w) * max(0, q.k)), no floating point involved on that side."""
+    q, k, w = synth.integer_indexer("pin_exact", 1, 64, 8, 128, -4, 4)
+    qi = q[0].to(torch.int64).numpy()
+    ki = k[0].to(torch.int64).numpy()
+    w4 = (w[0] * 4).to(torch.int64).numpy()
+    sc = indexer_scores(q[0], k[0], w[0])
+    for t in range(64):
+        dots = np.einsum("hd,sd->hs", qi[t], ki[:t + 1])
+        exact = (w4[t][:, None] * np.maximum(dots, 0)).sum(axis=0)
+        assert np.array_equal(sc[t, :t + 1].astype(np.float64) * 4, exact.astype(np.float64)), t
+    # fp8 form: codes are small integers, scales powers of two, so the same holds in units of 2^-8
+    q8, qs, k8, ks, w = synth.integer_indexer_e4m3("pin_exact8", 1, 48, 4, 128, -3, 3)
+    assert set(np.unique(e4m3_decode(q8.numpy()))) <= set(range(-3, 4))
+    sc8 = indexer_scores_fp8(q8[0].numpy(), qs[0].numpy(), k8[0].numpy(), ks[0].numpy(), w[0])
+    qv = e4m3_decode(q8[0].numpy()).astype(np.int64)
+    kv = e4m3_decode(k8[0].numpy()).astype(np.int64)
+    qsi = np.rint(qs[0].numpy() * 8).astype(np.int64)   # q_scale in units of 2^-3
+    ksi = np.rint(ks[0].numpy() * 8).astype(np.int64)
+    w4 = np.rint(w[0].numpy() * 4).astype(np.int64)
+    for t in range(48):
+        dots = np.einsum("hd,sd->hs", qv[t], kv[:t + 1])
+        exact = ksi[:t + 1] * (w4[t][:, None] * qsi[t][:, None] * np.maximum(dots, 0)).sum(axis=0)
+        assert np.array_equal(sc8[t, :t + 1].astype(np.float64) * 4 * 64, exact.astype(np.float64)), t

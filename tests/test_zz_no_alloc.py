@@ -20,21 +20,28 @@ from long_context_dsa_b200 import dsa, synth
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-# (name, n_q, H, d, k, fp8): the first has more work tiles than the array's CTA cap
-CASES = [("h32_k2048_3000", 3000, 32, 128, 2048, False),
-         ("tiny512", 512, 4, 64, 64, False),
-         ("fp8_h64_1100", 1100, 64, 128, 256, True)]
+# (name, B, n_q, n_kv, H, d, k, fp8): the first has more work tiles than the array's CTA cap; the
+# decode case (one query per sequence at the end of its cache) takes the split decode kernel,
+# whose partial lists and their merge also live in the array
+CASES = [("h32_k2048_3000", 1, 3000, 3000, 32, 128, 2048, False),
+         ("tiny512", 1, 512, 512, 4, 64, 64, False),
+         ("fp8_h64_1100", 1, 1100, 1100, 64, 128, 256, True),
+         ("decode_b8_4096", 8, 1, 4096, 32, 128, 2048, False)]
 
 
-def _inputs(name, L, H, d):
-    g = synth.StructuredIndexer("noalloc_" + name, 1, L, H, d, r=32, base_std=1.0, noise_std=0.2, seed=0)
-    return g.layer(0)
+def _inputs(name, B, n_q, L, H, d):
+    g = synth.StructuredIndexer("noalloc_" + name, B, L, H, d, r=32, base_std=1.0, noise_std=0.2, seed=0)
+    if n_q == L:
+        return g.layer(0)
+    q, w = g.queries(0, L - n_q, L)
+    return q, g.keys(0), w
 
 
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_noalloc_matches_workspace_entry_point_twice(case):
-    name, L, H, d, k, fp8 = case
-    q, kk, w = _inputs(name, L, H, d)
+    name, B, n_q, L, H, d, k, fp8 = case
+    q_pos0 = L - n_q
+    q, kk, w = _inputs(name, B, n_q, L, H, d)
     qs = ks = None
     dtype = dsa.DSA_BF16
     if fp8:
@@ -43,14 +50,15 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
         qs, ks = qs.to(DEV), ks.to(DEV)
         dtype = dsa.DSA_E4M3
     q, kk, w = q.to(DEV), kk.to(DEV), w.to(DEV)
-    ref = dsa.idx_score_topk(q, kk, w, k, q_scale=qs, k_scale=ks)
+    ref = dsa.idx_score_topk(q, kk, w, k, q_pos0=q_pos0, q_scale=qs, k_scale=ks)
     torch.cuda.synchronize()
     L_ = dsa.lib()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
     for call in range(2):
-        out = torch.full((1, L, k), -9, dtype=torch.int32, device=DEV)
-        rc = L_.idx_score_topk_noalloc(p(q), p(qs), p(kk), p(ks), p(w), dtype, 1, L, 0, L, H, d, k, p(out), stream)
+        out = torch.full((B, n_q, k), -9, dtype=torch.int32, device=DEV)
+        rc = L_.idx_score_topk_noalloc(p(q), p(qs), p(kk), p(ks), p(w), dtype, B, n_q, q_pos0, L, H, d, k, p(out),
+                                       stream)
         assert rc == dsa.DSA_OK, L_.dsa_last_error()
         torch.cuda.synchronize()
         # same kernel arithmetic as the workspace path: the selections agree exactly
