@@ -172,6 +172,57 @@ def attn_traffic():
     return round(per_pair * pairs)
 
 
+def stratified_random_indices(L_, k, dev, seed, rows_per_chunk=8192):
+    """Top-k-shaped index rows that defeat the workload's cross-query reuse: row t with t+1 > k
+    takes one uniformly random token from each of k equal strata of [0, t] (distinct, ascending);
+    shorter rows take every token, then -1.  Seeded, drawn on the device in row chunks."""
+    import torch
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    out = torch.empty((1, L_, k), dtype=torch.int32, device=dev)
+    i = torch.arange(k, device=dev, dtype=torch.int64)
+    for r0 in range(0, L_, rows_per_chunk):
+        r1 = min(L_, r0 + rows_per_chunk)
+        n = torch.arange(r0, r1, device=dev, dtype=torch.int64)[:, None] + 1      # tokens 0..t
+        lo = (i[None, :] * n) // k
+        hi = ((i[None, :] + 1) * n) // k
+        u = torch.rand((r1 - r0, k), generator=g, device=dev, dtype=torch.float64)
+        pick = lo + (u * (hi - lo).double()).long()
+        pick = torch.minimum(pick, hi - 1)
+        short = n <= k                                                               # every token, then -1
+        full = torch.where(i[None, :] < n, i[None, :], torch.full_like(pick, -1))
+        out[0, r0:r1] = torch.where(short, full, pick).int()
+    return out
+
+
+def attention_random_indices(layers, dev, stream, o_buf, ws, reps=3):
+    """The prefill workload's sparse attention (layer 0's Q/K/V, bf16 output, the bench's launch
+    configuration) on stratified random top-2048 rows instead of the indexer's selections: nearby
+    queries no longer share selections, so the gather leans on HBM instead of L2."""
+    import torch
+    from long_context_dsa_b200 import dsa
+
+    idx = stratified_random_indices(L, TOPK, dev, seed=77)
+    Lh = layers[0]
+    dsa.sparse_attn_topk(Lh["Q"], Lh["K"], Lh["V"], idx, o_dtype=torch.bfloat16, out=o_buf, workspace=ws,
+                         stream=stream)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dsa.sparse_attn_topk(Lh["Q"], Lh["K"], Lh["V"], idx, o_dtype=torch.bfloat16, out=o_buf, workspace=ws,
+                             stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    dsa.check_status(ws)
+    del idx
+    torch.cuda.empty_cache()
+    return sum(ts) / len(ts)
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     from long_context_dsa_b200 import dsa, replicas
@@ -231,6 +282,9 @@ def run_gpu(args, rank, world, local_rank):
                 idx_ms.append(evs[3 * l].elapsed_time(evs[3 * l + 1]))
             attn_ms.append(evs[3 * l + 1].elapsed_time(evs[3 * l + 2]))
 
+    # ---- the same attention on indices without cross-query reuse (HBM-bound gather)
+    rnd_ms = attention_random_indices(layers, dev, stream, layers[0]["O"], ws)
+
     # ---- all-F group (indexer ratio), untimed for `value`
     allf_evs = make_events()
     step(ALL_F)
@@ -257,6 +311,7 @@ def run_gpu(args, rank, world, local_rank):
     value = replicas.job_throughput(L, world, ms_per_step)
 
     abytes = attn_bytes()
+    dram = attn_traffic()
     iflops = indexer_flops()
     t_idx = 2 * iflops / (bf16_sus * 1e12)
     t_gather = N_LAYERS * abytes / (hbm * 1e9)
@@ -271,10 +326,24 @@ def run_gpu(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (q_I 1.6 GB, Q 1.6 GB per layer); no flush needed"},
         "roofline": {
             "bound": "hbm", "kernel": "sparse_attn_kernel (gathered K/V rows)",
-            "achieved": round(abytes / (attn_avg / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(abytes / (attn_avg / 1e3) / 1e9 / hbm, 4), "traffic": attn_traffic(),
+            "achieved": round(dram / (attn_avg / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(dram / (attn_avg / 1e3) / 1e9 / hbm, 4), "traffic": dram,
             "peak_source": f"{peak_src} hbm_gbs",
-            "algorithmic_bytes_per_launch": abytes, "avg_launch_ms": round(attn_avg, 3)},
+            "achieved_basis": "DRAM bytes per launch (ncu dram__bytes_read+write of the profiled tail case, "
+                              "scaled by selected (query, token) pairs) / average launch time in the timed region",
+            "algorithmic_bytes_per_launch": abytes, "avg_launch_ms": round(attn_avg, 3),
+            "gathered_gbs_equiv": round(abytes / (attn_avg / 1e3) / 1e9, 1),
+            "gathered_frac_equiv": round(abytes / (attn_avg / 1e3) / 1e9 / hbm, 4),
+            "gathered_note": "algorithmic gathered bytes (sum_t min(k,t+1) x Hkv x 2d x 2 B) / launch time: above "
+                             "HBM peak because nearby queries select the same tokens and L2 serves the repeats; "
+                             "this kernel is bound by gather latency, not by DRAM"},
+        "attention_random_indices": {
+            "kernel": "sparse_attn_kernel, same shape and launch configuration, stratified random top-2048 rows",
+            "avg_launch_ms": round(rnd_ms, 3),
+            "achieved": round(abytes / (rnd_ms / 1e3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(abytes / (rnd_ms / 1e3) / 1e9 / hbm, 4),
+            "note": "each token is still gathered by ~2000 queries over the launch, so L2 keeps part of the "
+                    "410 MB K/V; with no shared selections between neighbours the DRAM share is far higher"},
         "indexer_roofline": {
             "bound": "tensor", "kernel": "indexer_topk_kernel (fused scores + top-k)",
             "achieved": round(iflops / (idx_avg / 1e3) / 1e12, 1), "peak": bf16_sus, "unit": "TFLOP/s",
@@ -285,7 +354,9 @@ def run_gpu(args, rank, world, local_rank):
         "step_roofline": {"t_indexer_s": round(t_idx, 4), "t_gather_s": round(t_gather, 4),
                           "bound_s": round(step_roof_s, 4),
                           "frac": round(step_roof_s / (ms_per_step / 1e3), 4),
-                          "note": "max(indexer FLOPs at tensor peak, gathered bytes at HBM peak)"},
+                          "note": "the north star's bound: max(indexer FLOPs at tensor peak, gathered bytes at HBM "
+                                  "peak); the gathered bytes are largely L2 hits here (see roofline), so this bound "
+                                  "is not tight and a fraction near 1 does not mean the step is at its limit"},
         "index_sharing": {"all_f_step_ms": round(allf_step, 3), "shared_step_ms": round(ms_per_step, 3),
                           "all_f_indexer_ms": round(sum(allf_idx), 3),
                           "shared_indexer_ms": round(sum(idx_ms) / args.steps, 3),
@@ -590,6 +661,36 @@ def run_profile_paged(args):
     by = B * TOPK * HKV * DH * 2          # K and V codes gathered (bf16: twice this)
     print(json.dumps({"case": "profile_paged", "bf16_ms": min(t_b), "bf16_gathered_gbs": 2 * by / min(t_b) / 1e6,
                       "fp8_ms": min(t_8), "fp8_gathered_gbs": by / min(t_8) / 1e6}))
+
+
+def run_profile_latent(args):
+    """Small latent-attention case for ncu captures: 1024 query rows with 64 heads against a
+    262144-token latent cache (302 MB, larger than L2), stratified random top-2048 rows, bf16
+    output -- the tensor-core latent kernel (one unit per row)."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    dev = torch.device("cuda", 0)
+    n_kv, nq, hq = 1 << 18, 1024, 64
+    Q, KV, _ = synth.attention_inputs("proflat", 0, 1, nq, n_kv, hq, 1, 576, None, device=dev, seed=8)
+    idx = stratified_random_indices(n_kv, TOPK, dev, seed=8)[:, n_kv - nq:].contiguous()
+    O = torch.empty((1, nq, hq, 512), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(dsa.sparse_attn_topk_workspace_size(1, nq, n_kv, hq, 1, 576, 512, TOPK), dtype=torch.uint8,
+                     device=dev)
+    ts = []
+    for it in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dsa.sparse_attn_topk(Q, KV, None, idx, d_v=512, o_dtype=torch.bfloat16, out=O, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    dsa.check_status(ws)
+    by = nq * TOPK * 576 * 2
+    fl = nq * TOPK * hq * 2 * (576 + 512)
+    t = min(ts)
+    print(json.dumps({"case": "profile_latent", "ms": t, "gathered_gbs": by / t / 1e6, "tflops": fl / t / 1e9}))
 
 
 def run_decode(args, dev):
@@ -976,6 +1077,232 @@ def run_ctx1m(args, dev):
             "full_prefill_estimate_tok_per_s": round(L1 / est_s, 1)}
 
 
+def run_prefill16k(args, dev):
+    """The 16K-token prefill group: L=16384, batch 1, 4 layers FSSS, H_I=64 d_I=128 bf16 indexer,
+    top-2048, attention 32 query / 32 KV heads (MHA), d=128, bf16 output."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    L2, H2, HQ2, HKV2, pat = 16384, 64, 32, 32, "FSSS"
+    gen = synth.StructuredIndexer("prefill16k", 1, L2, H2, D_I, r=32, base_std=1.0, noise_std=0.2, device=dev,
+                                  seed=6000)
+    layers = []
+    for l in range(4):
+        Lh = {}
+        Lh["q_I"], Lh["k_I"], Lh["w"] = gen.layer(l)
+        Lh["Q"], Lh["K"], Lh["V"] = synth.attention_inputs("prefill16k", l, 1, L2, L2, HQ2, HKV2, DH, DH,
+                                                           device=dev, seed=6000)
+        Lh["O"] = torch.empty((1, L2, HQ2, DH), dtype=torch.bfloat16, device=dev)
+        layers.append(Lh)
+    del gen
+    shape = dsa.group_shape(1, L2, 0, L2, H2, D_I, HQ2, HKV2, DH, DH, TOPK, o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((1, L2, TOPK), dtype=torch.int32, device=dev))
+    sel = [dsa.idx_score_topk(layers[l]["q_I"], layers[l]["k_I"], layers[l]["w"], TOPK) for l in (0, 1)]
+    overlap = round(float(dsa.idx_overlap(sel[0][:, TOPK:].contiguous(), sel[1][:, TOPK:].contiguous()).double().mean().item())
+                    / TOPK, 4)
+    del sel
+    for _ in range(3):
+        dsa.layer_group_forward(shape, layers, pat, cache, workspace=ws)
+    torch.cuda.synchronize()
+    n = 5
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(12)]
+    for e in evs:
+        e.record()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(n):
+        dsa.layer_group_forward(shape, layers, pat, cache, workspace=ws, events=evs if i == n - 1 else None)
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b) / n
+    idx_ms = evs[0].elapsed_time(evs[1])
+    att_ms = [evs[3 * l + 1].elapsed_time(evs[3 * l + 2]) for l in range(4)]
+    hbm, _, bf16_sus, _ = peaks()
+    iflops = 2 * H2 * D_I * L2 * (L2 + 1) // 2
+    abytes = gathered_rows(L2, TOPK) * HKV2 * 2 * DH * 2
+    roof_s = iflops / (bf16_sus * 1e12) + 4 * abytes / (hbm * 1e9)
+    del layers
+    torch.cuda.empty_cache()
+    return {"workload": f"prefill L={L2}, batch 1, 4 layers {pat}, indexer H_I={H2} d_I={D_I} bf16 top-{TOPK}, "
+                        f"attention MHA {HQ2}Q/{HKV2}KV d={DH} bf16, bf16 output",
+            "tok_per_s": round(L2 / (ms / 1e3), 1), "ms_per_step": round(ms, 3),
+            "indexer_ms": round(idx_ms, 3),
+            "indexer_tflops": round(iflops / (idx_ms / 1e3) / 1e12, 1),
+            "attention_ms_per_layer": round(sum(att_ms) / 4, 3),
+            "attention_gathered_gbs": round(abytes / (sum(att_ms) / 4 / 1e3) / 1e9, 1),
+            "roofline_ms": round(roof_s * 1e3, 2),
+            "roofline_tok_per_s": round(L2 / roof_s, 1),
+            "roofline_note": "indexer FLOPs at sustained bf16 + gathered bytes at HBM peak; the 268 MB K/V of a "
+                             "layer is largely L2-resident, so the gather can beat its HBM time",
+            "adjacent_layer_overlap": overlap}
+
+
+def _ctx1m_caches(dev, n_kv, n_layers=N_LAYERS, seed=3000):
+    """The 1M-context caches: fp8 indexer keys (+ per-token scales) of the F layers and one latent
+    [1, n_kv, 576] bf16 cache per layer."""
+    import torch
+    from long_context_dsa_b200 import synth
+
+    gen = synth.StructuredIndexer("ctx1m", 1, n_kv, 64, D_I, r=32, base_std=1.0, noise_std=SIGMA_1M, device=dev,
+                                  seed=seed)
+    keys = {}
+    for l in range(n_layers):
+        if PATTERN[l] == "F":
+            keys[l] = synth.quantize_e4m3_rows(gen.keys(l))
+    lat = []
+    for l in range(n_layers):
+        _, KV, _ = synth.attention_inputs("ctx1m", l, 1, 1, n_kv, 64, 1, 576, None, device=dev, seed=seed)
+        lat.append(KV)
+        torch.cuda.empty_cache()
+    return gen, keys, lat
+
+
+def run_decode1m(args, dev):
+    """Decode after the 1M-token prefill: 32 steps, batch 1, the new token at positions 1048576 ..
+    1048607 (the cache grows from 1048577 to 1048608 tokens); 8 layers FSSSFSSS, fp8 indexer H_I=64
+    d_I=128 top-2048 (split decode kernel), latent attention 64 heads (split ranges + merge)."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    L1, steps, H1, HQ1 = 1 << 20, 32, 64, 64
+    n_max = L1 + steps
+    gen, keys, lat = _ctx1m_caches(dev, n_max)
+    qi = {}
+    for l in keys:
+        q, w = gen.queries(l, L1, n_max)                     # the 32 decode tokens' indexer queries
+        q8, qs = synth.quantize_e4m3_rows(q)
+        qi[l] = (q8, qs, w)
+    del gen
+    Qd = [synth.normal((1, steps, HQ1, 576), synth.seed_for(3000, "dec1m", l, "Q"), dev, dtype=torch.bfloat16)
+          for l in range(N_LAYERS)]
+    O = torch.empty((1, 1, HQ1, 512), dtype=torch.bfloat16, device=dev)
+    shape0 = dsa.group_shape(1, 1, n_max - 1, n_max, H1, D_I, HQ1, 1, 576, 512, TOPK, idx_dtype=dsa.DSA_E4M3,
+                             o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape0), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((1, 1, TOPK), dtype=torch.int32, device=dev))
+
+    def step(s, evs=None):
+        n_kv = L1 + s + 1
+        shape = dsa.group_shape(1, 1, n_kv - 1, n_kv, H1, D_I, HQ1, 1, 576, 512, TOPK, idx_dtype=dsa.DSA_E4M3,
+                                o_dtype=dsa.DSA_BF16)
+        layers = []
+        for l in range(N_LAYERS):
+            Lh = {"Q": Qd[l][:, s:s + 1], "K": lat[l][:, :n_kv], "V": None, "O": O}
+            if l in keys:
+                q8, qs, w = qi[l]
+                Lh.update(q_I=q8[:, s:s + 1], q_scale=qs[:, s:s + 1], w=w[:, s:s + 1],
+                          k_I=keys[l][0][:, :n_kv], k_scale=keys[l][1][:, :n_kv])
+            layers.append(Lh)
+        return dsa.layer_group_forward(shape, layers, PATTERN, cache, workspace=ws, events=evs)
+
+    for s in range(3):
+        step(s)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3 * N_LAYERS)] for _ in range(steps)]
+    for es in evs:
+        for e in es:
+            e.record()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(steps):
+        step(s, evs[s])
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b) / steps
+    idx_ms = sum(es[3 * l].elapsed_time(es[3 * l + 1]) for es in evs for l in range(N_LAYERS)) / steps
+    att_ms = sum(es[3 * l + 1].elapsed_time(es[3 * l + 2]) for es in evs for l in range(N_LAYERS)) / steps
+    hbm = peaks()[0]
+    n_f = PATTERN.count("F")
+    kbytes = n_f * (L1 + steps // 2) * (D_I + 4)            # fp8 keys + fp32 scales per F layer
+    abytes = N_LAYERS * TOPK * 576 * 2                      # the selected latent rows of every layer
+    bound_s = (kbytes + abytes) / (hbm * 1e9)
+    del lat, keys, qi, Qd
+    torch.cuda.empty_cache()
+    return {"workload": f"{steps} decode steps after a {L1}-token prefill, batch 1, 8 layers {PATTERN}, fp8 e4m3 "
+                        f"indexer H_I={H1} d_I={D_I} top-{TOPK}, latent attention 576/512 with {HQ1} heads",
+            "tok_per_s": round(1e3 / ms, 1), "ms_per_step": round(ms, 4),
+            "indexer_ms_per_step": round(idx_ms, 4), "attention_ms_per_step": round(att_ms, 4),
+            "hbm_bound_ms_per_step": round(bound_s * 1e3, 4),
+            "frac_of_hbm_bound": round(bound_s * 1e3 / ms, 4),
+            "bound_note": "fp8 keys + scales of the 2 F layers and 2048 latent rows of each of 8 layers, read "
+                          "once at measured HBM bandwidth"}
+
+
+def run_ctx1m_full(args, dev):
+    """The whole 1M-token chunked prefill, measured: 128 chunks of 8192 query rows, each chunk one
+    layer_group_forward over 8 layers FSSSFSSS (fp8 indexer H_I=64 on the 2 F layers, latent attention
+    with 64 heads on all 8) against the caches up to the chunk's end.  Keys and latent caches are the
+    full 1M-token tensors; every chunk's indexer queries are its own rows; the attention queries of one
+    chunk per layer are reused by every chunk (they set no control flow)."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    L1, C, H1, HQ1 = 1 << 20, 8192, 64, 64
+    n_chunks = L1 // C
+    gen, keys, lat = _ctx1m_caches(dev, L1)
+    qi = {}
+    for l in keys:
+        q8 = torch.empty((1, L1, H1, D_I), dtype=torch.uint8, device=dev)
+        qs = torch.empty((1, L1, H1), dtype=torch.float32, device=dev)
+        for c in range(n_chunks):
+            q, _ = gen.queries(l, c * C, (c + 1) * C)
+            q8[:, c * C:(c + 1) * C], qs[:, c * C:(c + 1) * C] = synth.quantize_e4m3_rows(q)
+        qi[l] = (q8, qs, gen.w.contiguous())
+    del gen
+    torch.cuda.empty_cache()
+    Qc = [synth.normal((1, C, HQ1, 576), synth.seed_for(3000, "ctx1m_full", l, "Q"), dev, dtype=torch.bfloat16)
+          for l in range(N_LAYERS)]
+    Oc = [torch.empty((1, C, HQ1, 512), dtype=torch.bfloat16, device=dev) for _ in range(N_LAYERS)]
+    shape_max = dsa.group_shape(1, C, L1 - C, L1, H1, D_I, HQ1, 1, 576, 512, TOPK, idx_dtype=dsa.DSA_E4M3,
+                                o_dtype=dsa.DSA_BF16)
+    ws = torch.zeros(dsa.layer_group_forward_workspace_size(shape_max), dtype=torch.uint8, device=dev)
+    cache = dsa.IndexCache(torch.empty((1, C, TOPK), dtype=torch.int32, device=dev))
+
+    def chunk(c, evs=None):
+        p0, n_kv = c * C, (c + 1) * C
+        shape = dsa.group_shape(1, C, p0, n_kv, H1, D_I, HQ1, 1, 576, 512, TOPK, idx_dtype=dsa.DSA_E4M3,
+                                o_dtype=dsa.DSA_BF16)
+        layers = []
+        for l in range(N_LAYERS):
+            Lh = {"Q": Qc[l], "K": lat[l][:, :n_kv], "V": None, "O": Oc[l]}
+            if l in qi:
+                q8, qs, w = qi[l]
+                Lh.update(q_I=q8[:, p0:n_kv], q_scale=qs[:, p0:n_kv], w=w[:, p0:n_kv],
+                          k_I=keys[l][0][:, :n_kv], k_scale=keys[l][1][:, :n_kv])
+            layers.append(Lh)
+        return dsa.layer_group_forward(shape, layers, PATTERN, cache, workspace=ws, events=evs)
+
+    chunk(0)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3 * N_LAYERS)] for _ in range(n_chunks)]
+    for es in evs:
+        for e in es:
+            e.record()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for c in range(n_chunks):
+        chunk(c, evs[c])
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b)
+    idx_ms = sum(es[3 * l].elapsed_time(es[3 * l + 1]) for es in evs for l in range(N_LAYERS))
+    att_ms = sum(es[3 * l + 1].elapsed_time(es[3 * l + 2]) for es in evs for l in range(N_LAYERS))
+    iflops = PATTERN.count("F") * 2 * H1 * D_I * L1 * (L1 + 1) // 2
+    abytes = N_LAYERS * gathered_rows(L1, TOPK) * 576 * 2
+    del lat, keys, qi, Qc, Oc
+    torch.cuda.empty_cache()
+    return {"workload": f"{L1}-token chunked prefill in {n_chunks} chunks of {C}, 8 layers {PATTERN}, fp8 e4m3 "
+                        f"indexer H_I={H1} d_I={D_I} top-{TOPK}, latent attention 576/512 with {HQ1} heads",
+            "seconds": round(ms / 1e3, 3), "tok_per_s": round(L1 / (ms / 1e3), 1),
+            "indexer_s": round(idx_ms / 1e3, 3), "attention_s": round(att_ms / 1e3, 3),
+            "indexer_fp8_tflops": round(iflops / (idx_ms / 1e3) / 1e12, 1),
+            "attention_gathered_gbs": round(abytes / (att_ms / 1e3) / 1e9, 1)}
+
+
 def run_cp(args, rank, world, local_rank):
     """Context-parallel prefill of ONE 200K-token sequence split over the ranks (strong
     scaling): every rank owns two zig-zag blocks of query rows, the keys (k_I of the F
@@ -1058,7 +1385,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench",
                     choices=["bench", "profile", "profile_paged", "decode", "decode_mha", "ctx1m", "mtp", "paged",
-                             "cp"],
+                             "prefill16k", "decode1m", "ctx1m_full", "profile_latent", "cp"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m / ...: only "
                          "that extra measurement, printed as one JSON line; cp: one 200K sequence split over "
                          "the torchrun ranks (context-parallel prefill, strong scaling)")
@@ -1069,11 +1396,16 @@ def main():
     if args.case == "profile_paged":
         run_profile_paged(args)
         return
-    if args.case in ("decode", "decode_mha", "ctx1m", "mtp", "paged"):
+    if args.case == "profile_latent":
+        run_profile_latent(args)
+        return
+    extra_cases = {"decode": run_decode, "decode_mha": run_decode_mha, "ctx1m": run_ctx1m, "mtp": run_mtp,
+                   "paged": run_paged, "prefill16k": run_prefill16k, "decode1m": run_decode1m,
+                   "ctx1m_full": run_ctx1m_full}
+    if args.case in extra_cases:
         import torch
         dev = torch.device("cuda", 0)
-        fn = {"decode": run_decode, "decode_mha": run_decode_mha, "ctx1m": run_ctx1m, "mtp": run_mtp,
-              "paged": run_paged}[args.case]
+        fn = extra_cases[args.case]
         print(json.dumps({"case": args.case, **fn(args, dev)}), flush=True)
         return
 
@@ -1118,6 +1450,9 @@ def main():
         out["multi_token_decode"] = run_mtp(args, dev)
         out["paged_decode"] = run_paged(args, dev)
         out["context_1m_tail_chunk"] = run_ctx1m(args, dev)
+        out["prefill_16k"] = run_prefill16k(args, dev)
+        out["decode_after_1m"] = run_decode1m(args, dev)
+        out["context_1m_full_prefill"] = run_ctx1m_full(args, dev)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -36,6 +36,7 @@ cudaError_t launch_overlap_count(const int* a, const int* b, long long rows, int
                                  cudaStream_t stream);
 void greedy_pattern(const double* ov, int n, int n_f, char* out);
 size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms);
+size_t sparse_attn_latent_part_bytes(int B, int n_q, int Hq, int topk, int num_sms);
 cudaError_t launch_indexer(const void* q, const float* q_scale, const void* k, const float* k_scale,
                            const float* w, int dtype, int B, int n_q, int q_pos0, int n_kv, int H, int d,
                            int topk, int* idx_out, float* scores_out, void* ws, size_t ws_bytes, int num_sms,
@@ -320,6 +321,11 @@ int sparse_attn_topk_workspace_size(int B, int n_q, int n_kv, int Hq, int Hkv, i
         int rc = sm_count(&sms);
         if (rc) return rc;
         part = sparse_attn_part_bytes(B, n_q, Hq, Hkv, d_qk, topk, sms);
+    } else if (d_qk == 576 && d_v == 512 && Hkv == 1) {  // the latent form
+        int sms;
+        int rc = sm_count(&sms);
+        if (rc) return rc;
+        part = sparse_attn_latent_part_bytes(B, n_q, Hq, topk, sms);
     }
     *bytes = kWsHeaderBytes + part;
     return DSA_OK;

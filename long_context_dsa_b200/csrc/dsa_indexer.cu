@@ -521,8 +521,9 @@ cudaError_t launch_t(const void* q, const float* q_scale, const void* k, const f
 
 bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype);
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen);
-cudaError_t launch_indexer_decode(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int H,
-                                  int topk, int* idx_out, void* ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_indexer_decode(const void* q, const float* q_scale, const void* k, const float* k_scale,
+                                  const float* w, int dtype, int B, int q_pos0, int n_kv, int H, int topk,
+                                  int* idx_out, void* ws, int num_sms, cudaStream_t stream);
 
 size_t indexer_workspace_bytes(int B, int n_q, int q_pos0, int n_kv, int H, int d, int topk, int dtype,
                                int num_sms) {
@@ -540,7 +541,8 @@ cudaError_t launch_indexer(const void* q, const float* q_scale, const void* k, c
     (void)ws_bytes;
     // one query per sequence: the split decode kernel (the selection path only)
     if (!scores_out && indexer_decode_supported(B, n_q, q_pos0, n_kv, H, d, topk, dtype))
-        return launch_indexer_decode(q, k, w, B, q_pos0, n_kv, H, topk, idx_out, ws, num_sms, stream);
+        return launch_indexer_decode(q, q_scale, k, k_scale, w, dtype, B, q_pos0, n_kv, H, topk, idx_out, ws, num_sms,
+                                     stream);
 #define DSA_IDX_CASE(HH, DD, F8)                                                                              \
     if (H == HH && d == DD && (dtype == DSA_E4M3) == F8)                                                     \
         return launch_t<HH, DD, F8>(q, q_scale, k, k_scale, w, B, n_q, q_pos0, n_kv, topk, idx_out, scores_out, ws, \

@@ -30,13 +30,17 @@ namespace dsa {
 cudaError_t launch_topk_merge_pairs(const uint32_t* keys, const int* idxs, int rows, int len, int k, int* out,
                                     WsHeader* hdr, int num_sms, cudaStream_t stream, int n_tok);
 
-template <int H>
+template <int H, bool FP8>
 struct DecCfg {
     static constexpr int N = H;              // accumulator columns: one query's heads
     static constexpr int NACC = 512 / N;     // accumulators in flight
-    static constexpr int STAGES = 4;
-    static constexpr int A_STAGE = 128 * 256;  // 128 keys x 128 bf16
-    static constexpr int B_BYTES = N * 256;    // the query's H rows x 128 bf16
+    static constexpr int ROWB = FP8 ? 128 : 256;  // bytes per key / query-head row (d_I = 128)
+    static constexpr int KB = ROWB / 128;         // 128-byte swizzle blocks per row
+    static constexpr int KSTEPS = ROWB / 32;      // MMA K-steps of 32 bytes
+    static constexpr int BOX_X = FP8 ? 128 : 64;  // elements per 128-byte TMA box row
+    static constexpr int STAGES = FP8 ? 8 : 4;    // the same 128 KB of keys in flight either way
+    static constexpr int A_STAGE = 128 * ROWB;    // 128 keys
+    static constexpr int B_BYTES = N * ROWB;      // the query's H rows
     static constexpr int CAP = kCandCap;       // candidate buffer of the unit's row (shared memory)
     static constexpr int THREADS = 192;        // warps 0-3 epilogue, 4 producer, 5 MMA
     static constexpr int OFF_B = 0;
@@ -56,6 +60,8 @@ struct DecCfg {
 
 struct DecParams {
     const float* w;
+    const float* q_scale;   // [B, H] (e4m3 only): folded into w
+    const float* k_scale;   // [B, n_kv] (e4m3 only): multiplies each key's score
     const int* seq_lens;    // [B] cache length of each sequence, or NULL: every sequence has q_pos0 + 1 keys
     const int* page_table;  // [B, max_pages] physical page of each logical page, or NULL: contiguous [B, n_kv]
     int page_size, max_pages, num_pages;
@@ -65,11 +71,11 @@ struct DecParams {
     WsHeader* hdr;
 };
 
-template <int H>
+template <int H, bool FP8>
 __global__ void __launch_bounds__(192, 1)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                           const DecParams p) {
-    using C = DecCfg<H>;
+    using C = DecCfg<H, FP8>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     unsigned char* sB = smem + C::OFF_B;
@@ -148,21 +154,24 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t it = 0, wt = 0;
             bool ok = true;
             int pend_q = -1;
+            const bool withhold = test_withhold_tile(p.hdr);  // timeout test: first key tile never sent
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++wt) {
                 int b, j0, j1, len;
                 unit_range(u, b, j0, j1, len);
                 if (wt > 0 && !mbar_wait(q_empty, (wt - 1) & 1)) { ok = false; break; }
                 mbar_arrive_expect_tx(q_full, C::B_BYTES);
-                for (int kb = 0; kb < 2; ++kb) tc::tma_load_2d(sB + kb * H * 128, &tmap_q, kb * 64, b * H, q_full);
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tc::tma_load_2d(sB + kb * H * 128, &tmap_q, kb * C::BOX_X, b * H, q_full);
                 pend_q = static_cast<int>(wt);
                 for (int j = j0; j < j1; ++j, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t rr = it / C::STAGES;
                     if (rr > 0 && !mbar_wait(&kv_empty[s], (rr - 1) & 1)) { ok = false; break; }
+                    if (withhold && it == 0) continue;  // nothing issued: the waits on this stage run out
                     mbar_arrive_expect_tx(&kv_full[s], C::A_STAGE);
-                    if (!p.page_table) {
-                        for (int kb = 0; kb < 2; ++kb)
-                            tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128, &tmap_k, kb * 64,
+                    if (FP8 || !p.page_table) {  // (the fp8 form is built for contiguous caches only)
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tc::tma_load_2d(sA + s * C::A_STAGE + kb * 128 * 128, &tmap_k, kb * C::BOX_X,
                                             b * p.n_kv + j * 128, &kv_full[s]);
                     } else {
                         // the tile's 128 keys page by page (rows = pieces of min(page, 128) keys; the
@@ -194,7 +203,7 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 5) {
         // ================================================== MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::make_idesc(1, 1, 128, C::N);
+            constexpr uint32_t idesc = FP8 ? tc::make_idesc(0, 0, 128, C::N) : tc::make_idesc(1, 1, 128, C::N);
             uint32_t it = 0, wt = 0, ua = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++wt) {
@@ -212,10 +221,13 @@ __global__ void __launch_bounds__(192, 1)
                     tc::fence_after_sync();
                     const uint32_t a0 = smem_u32(sA + s * C::A_STAGE);
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
+                    for (int ks = 0; ks < C::KSTEPS; ++ks) {
                         const uint64_t ad = tc::make_sdesc_sw128(a0 + (ks >> 2) * (128 * 128) + (ks & 3) * 32);
                         const uint64_t bd = tc::make_sdesc_sw128(b0 + (ks >> 2) * (H * 128) + (ks & 3) * 32);
-                        tc::mma_f16(tmem_base + a * C::N, ad, bd, idesc, ks > 0);
+                        if (FP8)
+                            tc::mma_f8(tmem_base + a * C::N, ad, bd, idesc, ks > 0);
+                        else
+                            tc::mma_f16(tmem_base + a * C::N, ad, bd, idesc, ks > 0);
                     }
                     tc::mma_commit(&acc_full[a]);
                     tc::mma_commit(&kv_empty[s]);
@@ -241,7 +253,11 @@ __global__ void __launch_bounds__(192, 1)
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int b, j0, j1, len;
             unit_range(u, b, j0, j1, len);
-            if (tid < H) ws[tid] = p.w[static_cast<size_t>(b) * H + tid];
+            if (tid < H) {  // head weights (fp8: folded with the query's per-head scale)
+                float wv = p.w[static_cast<size_t>(b) * H + tid];
+                if (FP8) wv *= p.q_scale[static_cast<size_t>(b) * H + tid];
+                ws[tid] = wv;
+            }
             if (tid == 0) topk_row_init(st);
             grp.sync();
             int cnt = 0;
@@ -277,6 +293,7 @@ __global__ void __launch_bounds__(192, 1)
                     *wg_abort = 1;
                 }
                 const int s_key = j * 128 + tid;
+                if (FP8) sc_v *= (s_key < len) ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s_key] : 0.f;
                 const uint32_t key = score_key(sc_v);
                 const uint32_t tk = st->thr_key;
                 const bool adm = got & (s_key < len) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
@@ -322,8 +339,8 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
-    // [rows, 128] bf16, 128-byte swizzled boxes of 64 columns x box_rows
+bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows, bool fp8) {
+    // [rows, 128] bf16 or e4m3, 128-byte swizzled boxes of 128 bytes x box_rows
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
         void* ptr = nullptr;
@@ -335,10 +352,10 @@ bool make_map_dec(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_
         fn = reinterpret_cast<EncodeTiledFn>(ptr);
     }
     cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint64_t strides[1] = {fp8 ? 128u : 256u};
+    cuuint32_t box[2] = {fp8 ? 128u : 64u, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -369,20 +386,25 @@ struct DecCache {
     int page_size, max_pages, num_pages, max_len;
 };
 
-template <int H>
-cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int topk,
-                         const DecCache& pc, int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
-    using C = DecCfg<H>;
+template <int H, bool FP8>
+cudaError_t launch_dec_t(const void* q, const float* q_scale, const void* k, const float* k_scale, const float* w,
+                         int B, int q_pos0, int n_kv, int topk, const DecCache& pc, int* idx_out, void* ws,
+                         int num_sms, cudaStream_t stream) {
+    using C = DecCfg<H, FP8>;
     CUtensorMap mq, mk;
     const bool paged = pc.page_table != nullptr;
+    if (FP8 && paged) return cudaErrorNotSupported;
     const uint64_t krows = paged ? static_cast<uint64_t>(pc.num_pages) * pc.page_size : static_cast<uint64_t>(B) * n_kv;
-    if (!make_map_dec(&mq, q, static_cast<uint64_t>(B) * H, H) ||
-        !make_map_dec(&mk, k, krows, paged ? static_cast<uint32_t>(pc.page_size < 128 ? pc.page_size : 128) : 128))
+    if (!make_map_dec(&mq, q, static_cast<uint64_t>(B) * H, H, FP8) ||
+        !make_map_dec(&mk, k, krows, paged ? static_cast<uint32_t>(pc.page_size < 128 ? pc.page_size : 128) : 128,
+                      FP8))
         return cudaErrorInvalidValue;
     const int max_len = pc.seq_lens ? pc.max_len : q_pos0 + 1;
     const int nkt = (max_len + 127) / 128;
     DecParams p;
     p.w = w;
+    p.q_scale = q_scale;
+    p.k_scale = k_scale;
     p.seq_lens = pc.seq_lens;
     p.page_table = pc.page_table;
     p.page_size = pc.page_size;
@@ -399,7 +421,7 @@ cudaError_t launch_dec_t(const void* q, const void* k, const float* w, int B, in
     const size_t parts = static_cast<size_t>(B) * p.splits * topk;
     p.part_key = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kWsHeaderBytes);
     p.part_idx = reinterpret_cast<int*>(p.part_key + parts);
-    auto kern = indexer_decode_kernel<H>;
+    auto kern = indexer_decode_kernel<H, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int units = B * p.splits;
@@ -415,7 +437,8 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
     (void)B;
     (void)n_kv;
     (void)topk;
-    return n_q == 1 && d == 128 && dtype == DSA_BF16 && (H == 32 || H == 64) && q_pos0 + 1 >= 8 * 128;
+    return n_q == 1 && d == 128 && (dtype == DSA_BF16 || dtype == DSA_E4M3) && (H == 32 || H == 64) &&
+           q_pos0 + 1 >= 8 * 128;
 }
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen) {
@@ -426,11 +449,20 @@ size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, 
     return static_cast<size_t>(B) * splits * topk * 8;
 }
 
-cudaError_t launch_indexer_decode(const void* q, const void* k, const float* w, int B, int q_pos0, int n_kv, int H,
-                                  int topk, int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
+cudaError_t launch_indexer_decode(const void* q, const float* q_scale, const void* k, const float* k_scale,
+                                  const float* w, int dtype, int B, int q_pos0, int n_kv, int H, int topk,
+                                  int* idx_out, void* ws, int num_sms, cudaStream_t stream) {
     const DecCache none = {nullptr, nullptr, 0, 0, 0, 0};
-    if (H == 32) return launch_dec_t<32>(q, k, w, B, q_pos0, n_kv, topk, none, idx_out, ws, num_sms, stream);
-    if (H == 64) return launch_dec_t<64>(q, k, w, B, q_pos0, n_kv, topk, none, idx_out, ws, num_sms, stream);
+    const bool f8 = dtype == DSA_E4M3;
+#define DSA_DEC_CASE(HH, F8)                                                                                   \
+    if (H == HH && f8 == F8)                                                                                   \
+        return launch_dec_t<HH, F8>(q, q_scale, k, k_scale, w, B, q_pos0, n_kv, topk, none, idx_out, ws, num_sms, \
+                                    stream);
+    DSA_DEC_CASE(32, false)
+    DSA_DEC_CASE(64, false)
+    DSA_DEC_CASE(32, true)
+    DSA_DEC_CASE(64, true)
+#undef DSA_DEC_CASE
     return cudaErrorNotSupported;
 }
 
@@ -439,8 +471,12 @@ cudaError_t launch_indexer_decode_paged(const void* q, const void* k_pages, cons
                                         int max_pages, int H, int topk, int* idx_out, void* ws, int num_sms,
                                         cudaStream_t stream) {
     const DecCache pc = {seq_lens, page_table, page_size, max_pages, num_pages, max_len};
-    if (H == 32) return launch_dec_t<32>(q, k_pages, w, B, max_len - 1, 0, topk, pc, idx_out, ws, num_sms, stream);
-    if (H == 64) return launch_dec_t<64>(q, k_pages, w, B, max_len - 1, 0, topk, pc, idx_out, ws, num_sms, stream);
+    if (H == 32)
+        return launch_dec_t<32, false>(q, nullptr, k_pages, nullptr, w, B, max_len - 1, 0, topk, pc, idx_out, ws,
+                                       num_sms, stream);
+    if (H == 64)
+        return launch_dec_t<64, false>(q, nullptr, k_pages, nullptr, w, B, max_len - 1, 0, topk, pc, idx_out, ws,
+                                       num_sms, stream);
     return cudaErrorNotSupported;
 }
 

@@ -70,11 +70,15 @@ struct Cfg {
     static constexpr size_t SMEM = Q_BYTES + static_cast<size_t>(STAGES) * STAGE_BYTES + STAGES * CHUNK * 4;
 };
 
-template <int WARPS, bool OUT_BF16>
+// SPLIT: each (query row, head block) unit is cut into `splits` ranges of `cps` chunks (few
+// rows, e.g. one decode token: the ranges spread over the SMs); a range writes its unnormalised
+// O and its (max, sum) per head to `part` and latent_merge_kernel combines the ranges.
+template <int WARPS, bool OUT_BF16, bool SPLIT>
 __global__ void __launch_bounds__(WARPS * 32, 1)
     latent_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ KV,
                        const int* __restrict__ idx, int B, int n_q, int n_kv, int Hq, int topk, float scale_log2,
-                       void* __restrict__ O, IdxShare share, WsHeader* hdr) {
+                       void* __restrict__ O, int splits, int cps, float* __restrict__ part, IdxShare share,
+                       WsHeader* hdr) {
     using C = Cfg<WARPS>;
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char* sq = smem;
@@ -85,6 +89,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     const int nthr = WARPS * 32;
     const int hblocks = Hq / C::HB;
     const long long units = static_cast<long long>(B) * n_q * hblocks;
+    const long long items = SPLIT ? units * splits : units;
     const int nchunks = (topk + CHUNK - 1) / CHUNK;
 
     const int qn = lane >> 2, hc = 2 * (lane & 3);
@@ -94,7 +99,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     // Q^T B fragments via ldmatrix.x4 over two k-steps: rows = heads, 8-element column groups
     const int q_row = lane & 7, q_col = (lane >> 3) * 8;
 
-    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+    for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+        const long long u = SPLIT ? it / splits : it;
+        const int sp = SPLIT ? static_cast<int>(it % splits) : 0;
+        const int c0 = SPLIT ? sp * cps : 0;                       // this item's chunk range
+        const int c1 = SPLIT ? min(nchunks, c0 + cps) : nchunks;
         const long long row = u / hblocks;
         const int hb = static_cast<int>(u % hblocks);
         const long long b = row / n_q;
@@ -113,8 +122,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             }
         }
         auto issue = [&](int c) {
-            if (c < nchunks) {
-                const int s = c % STAGES;
+            if (c < c1) {
+                const int s = (c - c0) % STAGES;
                 if (threadIdx.x < CHUNK) {
                     const int kk = c * CHUNK + threadIdx.x;
                     int t = kk < topk ? __ldg(irow + kk) : -1;
@@ -143,12 +152,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
         const uint32_t qw = sq_s + (warp * 8 + q_row) * RS + q_col * 2;  // this lane's ldmatrix row of Q
 
 #pragma unroll
-        for (int c = 0; c < STAGES - 1; ++c) issue(c);
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = c0; c < c0 + STAGES - 1; ++c) issue(c);
+        for (int c = c0; c < c1; ++c) {
             issue(c + STAGES - 1);
             cp_async_wait<STAGES - 1>();
             __syncthreads();
-            const int s = c % STAGES;
+            const int s = (c - c0) % STAGES;
             const uint32_t kst = ring_s + s * C::STAGE_BYTES;
             const int* si = sidx + s * CHUNK;
             // ---- S^T = K Q^T over 36 k-steps (two per ldmatrix.x4 of Q)
@@ -214,6 +223,28 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) lrun[j] += __shfl_xor_sync(0xffffffffu, lrun[j], off);
         }
+        if (SPLIT) {
+            // unnormalised O^T and (max, sum) of this range, per head: [item][head][DV + 2]
+#pragma unroll
+            for (int dt = 0; dt < DV / 16; ++dt) {
+                const int d0 = dt * 16 + qn;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float* pp = part + (static_cast<size_t>(it) * C::HB + warp * 8 + hc + j) * (DV + 2);
+                    pp[d0] = o[dt][j];
+                    pp[d0 + 8] = o[dt][2 + j];
+                }
+            }
+            if (qn == 0) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float* pp = part + (static_cast<size_t>(it) * C::HB + warp * 8 + hc + j) * (DV + 2);
+                    pp[DV] = mrun[j];
+                    pp[DV + 1] = lrun[j];
+                }
+            }
+            continue;
+        }
         const float inv0 = lrun[0] > 0.f ? 1.f / lrun[0] : 0.f;
         const float inv1 = lrun[1] > 0.f ? 1.f / lrun[1] : 0.f;
 #pragma unroll
@@ -238,38 +269,132 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     }
 }
 
+// Combine the split ranges of each (query row, head block): for every head,
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s (a range that met only
+// skipped entries has m_s = -inf and drops out).  One block per unit, a warp per head at a
+// time; lane s holds range s's (m, l) (splits <= 32) and each lane owns DV/32 columns.
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(512)
+    latent_merge_kernel(const float* __restrict__ part, int HB, int hblocks, int splits, int Hq,
+                        void* __restrict__ O) {
+    const long long u = blockIdx.x;  // (row, head block)
+    const long long row = u / hblocks;
+    const int hb = static_cast<int>(u % hblocks);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t sstride = static_cast<size_t>(HB) * (DV + 2);
+    for (int h = warp; h < HB; h += 16) {
+        const float* p0 = part + (static_cast<size_t>(u) * splits * HB + h) * (DV + 2);
+        const float m = lane < splits ? __ldg(p0 + lane * sstride + DV) : -INFINITY;
+        const float l = lane < splits ? __ldg(p0 + lane * sstride + DV + 1) : 0.f;
+        float M = m;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+        float L = f * l;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        float acc[DV / 32];
+#pragma unroll
+        for (int i = 0; i < DV / 32; ++i) acc[i] = 0.f;
+        for (int s2 = 0; s2 < splits; ++s2) {
+            const float fs = __shfl_sync(0xffffffffu, f, s2);
+#pragma unroll
+            for (int i = 0; i < DV / 32; ++i) acc[i] += fs * __ldg(p0 + s2 * sstride + i * 32 + lane);
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const size_t ob = (static_cast<size_t>(row) * Hq + static_cast<size_t>(hb) * HB + h) * DV;
+#pragma unroll
+        for (int i = 0; i < DV / 32; ++i) {
+            if (OUT_BF16)
+                reinterpret_cast<__nv_bfloat16*>(O)[ob + i * 32 + lane] = __float2bfloat16_rn(acc[i] * inv);
+            else
+                reinterpret_cast<float*>(O)[ob + i * 32 + lane] = acc[i] * inv;
+        }
+    }
+}
+
+// Warps per CTA (8 query heads each) for Hq query heads.
+inline int warps_for(int Hq) { return Hq % 64 == 0 ? 8 : Hq % 32 == 0 ? 4 : Hq % 16 == 0 ? 2 : 1; }
+
+// Ranges per (row, head block) unit: 1 when the units alone fill every SM; otherwise enough to
+// give each SM about one item, at most 32 ranges and at least 2 chunks (32 keys) each.  Depends
+// only on the shape and the SM count, so the workspace query and the launch agree.
+inline int latent_splits(long long units, int nchunks, int num_sms, int* cps) {
+    int s = 1;
+    if (units < num_sms) {
+        s = static_cast<int>((num_sms + units - 1) / units);
+        const int most = nchunks / 2 > 1 ? nchunks / 2 : 1;
+        if (s > most) s = most;
+        if (s > 32) s = 32;
+    }
+    *cps = (nchunks + s - 1) / s;
+    return (nchunks + *cps - 1) / *cps;
+}
+
 template <int WARPS>
 cudaError_t launch_w(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv, int Hq, int topk,
                      float scale, void* O, bool out_bf16, IdxShare share, WsHeader* hdr, int num_sms,
                      cudaStream_t stream) {
     using Cf = Cfg<WARPS>;
-    auto kern = out_bf16 ? latent_attn_kernel<WARPS, true> : latent_attn_kernel<WARPS, false>;
+    const int hblocks = Hq / Cf::HB;
+    const long long units = static_cast<long long>(B) * n_q * hblocks;
+    const int nchunks = (topk + CHUNK - 1) / CHUNK;
+    int cps = nchunks;
+    const int splits = latent_splits(units, nchunks, num_sms, &cps);
+    auto kern = out_bf16 ? (splits > 1 ? latent_attn_kernel<WARPS, true, true> : latent_attn_kernel<WARPS, true, false>)
+                         : (splits > 1 ? latent_attn_kernel<WARPS, false, true> : latent_attn_kernel<WARPS, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cf::SMEM));
     if (e != cudaSuccess) return e;
-    const long long units = static_cast<long long>(B) * n_q * (Hq / Cf::HB);
+    const long long items = units * splits;
     long long grid = num_sms;
-    if (grid > units) grid = units;
+    if (grid > items) grid = items;
     if (grid < 1) grid = 1;
+    float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(hdr) + kWsHeaderBytes);
     kern<<<static_cast<int>(grid), WARPS * 32, Cf::SMEM, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(KV), idx, B, n_q, n_kv, Hq, topk,
-        scale * 1.4426950408889634f, O, share, hdr);
+        scale * 1.4426950408889634f, O, splits, cps, part, share, hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    if (out_bf16)
+        latent_merge_kernel<true><<<static_cast<unsigned>(units), 512, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
+    else
+        latent_merge_kernel<false><<<static_cast<unsigned>(units), 512, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
     return cudaGetLastError();
 }
 
 }  // namespace lat
 
+bool latent_tc_applies(int B, int n_q, int Hq, int num_sms);
+cudaError_t launch_latent_tc(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv, int Hq,
+                             int topk, float scale, void* O, bool out_bf16, IdxShare share, WsHeader* hdr,
+                             int num_sms, cudaStream_t stream);
+
+// Many query rows with heads in blocks of 64: the tensor-core kernel (dsa_latent_tc.cu).  Otherwise
+// (decode, a few rows, other head counts) the warp-MMA kernel above, with split ranges when the
+// rows alone cannot fill the GPU.
 cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
                                       int Hq, int topk, float scale, void* O, bool out_bf16, IdxShare share,
                                       WsHeader* hdr, int num_sms, cudaStream_t stream) {
-    if (Hq % 64 == 0)
-        return lat::launch_w<8>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
-    if (Hq % 32 == 0)
-        return lat::launch_w<4>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
-    if (Hq % 16 == 0)
-        return lat::launch_w<2>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
-    if (Hq % 8 == 0)
-        return lat::launch_w<1>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
-    return cudaErrorNotSupported;
+    if (latent_tc_applies(B, n_q, Hq, num_sms))
+        return launch_latent_tc(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
+    switch (lat::warps_for(Hq)) {
+        case 8: return lat::launch_w<8>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
+        case 4: return lat::launch_w<4>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
+        case 2: return lat::launch_w<2>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
+        default:
+            if (Hq % 8 != 0) return cudaErrorNotSupported;
+            return lat::launch_w<1>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
+    }
+}
+
+// Bytes of split-range state the latent attention needs beyond the status word.
+size_t sparse_attn_latent_part_bytes(int B, int n_q, int Hq, int topk, int num_sms) {
+    if (Hq < 8 || Hq % 8 != 0) return 0;
+    const int HB = 8 * lat::warps_for(Hq);
+    const long long units = static_cast<long long>(B) * n_q * (Hq / HB);
+    int cps = 0;
+    const int splits = lat::latent_splits(units, (topk + lat::CHUNK - 1) / lat::CHUNK, num_sms, &cps);
+    if (splits == 1) return 0;
+    return static_cast<size_t>(units) * splits * HB * (lat::DV + 2) * sizeof(float);
 }
 
 }  // namespace dsa

@@ -50,3 +50,16 @@ def test_context_parallel_plan_of_the_workload():
         work = [cp.indexer_work(p) for p in plans]
         assert sum(work) == L * (L + 1) // 2
         assert max(work) / (sum(work) / W) < 1.001
+
+
+def test_stratified_random_indices_are_causal_distinct_ascending(bench):
+    import numpy as np
+    idx = bench.stratified_random_indices(3000, 128, "cpu", 5, rows_per_chunk=1000)[0].numpy()
+    for t in range(0, 3000, 7):
+        n = min(128, t + 1)
+        row = idx[t]
+        assert np.all(row[n:] == -1)
+        assert np.all(np.diff(row[:n]) > 0) and row[0] >= 0 and row[n - 1] <= t
+        if t + 1 > 128:  # one token from each of the 128 strata of [0, t]
+            strata = (np.arange(128) * (t + 1)) // 128
+            assert np.all(row[:n] >= strata) and np.all(row[:n] < np.append(strata[1:], t + 1))

@@ -137,6 +137,13 @@ LATENT = [
     ("latent_h16_chunk_b2", 2, 100, 400, 500, 16, 300, None),
     ("latent_h8_k64", 1, 200, 0, 200, 8, 64, None),
     ("latent_h64_k2048", 1, 2600, 0, 2600, 64, 2048, 48),
+    # one query row per sequence (decode): few (row, head block) units, so each unit's index list
+    # is cut into ranges over the SMs and a second kernel merges them
+    ("latent_decode_b1_h64", 1, 1, 4999, 5000, 64, 2048, None),
+    ("latent_decode_b3_h16_k300", 3, 1, 999, 1000, 16, 300, None),
+    ("latent_decode_b2_h8_k37", 2, 1, 199, 200, 8, 37, None),
+    # rows shorter than k: most ranges hold only -1 entries and must drop out of the merge
+    ("latent_decode_short_h64", 2, 1, 99, 100, 64, 2048, None),
 ]
 
 
@@ -145,7 +152,8 @@ def test_latent_attention_matches_oracle(case):
     name, B, n_q, q_pos0, n_kv, Hq, k, sample = case
     Q, KV, _ = synth.attention_inputs(name, 0, B, n_q, n_kv, Hq, 1, 576, None)
     idx = _indices(n_kv, k, 8, q_pos0, n_q, B)
-    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(dsa.sparse_attn_topk_workspace_size(B, n_q, n_kv, Hq, 1, 576, 512, k), dtype=torch.uint8,
+                     device=DEV)
     O = dsa.sparse_attn_topk(Q.to(DEV), KV.to(DEV), None, torch.from_numpy(idx).to(DEV), d_v=512, workspace=ws)
     assert dsa.read_status(ws) == 0
     O = O.cpu().numpy()
