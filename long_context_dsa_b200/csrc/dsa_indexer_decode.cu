@@ -29,6 +29,9 @@ namespace dsa {
 
 cudaError_t launch_topk_merge_pairs(const uint32_t* keys, const int* idxs, int rows, int len, int k, int* out,
                                     WsHeader* hdr, int num_sms, cudaStream_t stream, int n_tok);
+size_t radix_topk_scratch_bytes(int rows, int n, int num_sms);
+cudaError_t launch_radix_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
+                              int num_sms, cudaStream_t stream);
 
 template <int H, bool FP8>
 struct DecCfg {
@@ -68,6 +71,7 @@ struct DecParams {
     int B, q_pos0, n_kv, topk, splits, tiles_per_split;
     uint32_t* part_key;  // [B * splits, topk]
     int* part_idx;       // [B * splits, topk]
+    uint32_t* score_keys;  // [B, q_pos0 + 1] order-preserving score keys (score mode), or NULL
     WsHeader* hdr;
 };
 
@@ -295,9 +299,14 @@ __global__ void __launch_bounds__(192, 1)
                 const int s_key = j * 128 + tid;
                 if (FP8) sc_v *= (s_key < len) ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s_key] : 0.f;
                 const uint32_t key = score_key(sc_v);
-                const uint32_t tk = st->thr_key;
-                const bool adm = got & (s_key < len) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
-                topk_append_warp(wkey, widx, cnt, key, s_key, adm, sub);
+                if (p.score_keys) {
+                    // score mode: the row's keys go to memory and a multi-CTA radix select picks the top-k
+                    if (got && s_key < len) p.score_keys[static_cast<size_t>(b) * (p.q_pos0 + 1) + s_key] = key;
+                } else {
+                    const uint32_t tk = st->thr_key;
+                    const bool adm = got & (s_key < len) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
+                    topk_append_warp(wkey, widx, cnt, key, s_key, adm, sub);
+                }
                 if (((j - j0) % CHECK) == CHECK - 1 || j == j1 - 1) {
                     if (lane == 0) st->cnt[warp] = cnt;
                     grp.sync();
@@ -317,6 +326,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             if (!ok) break;
+            if (p.score_keys) continue;
             if (lane == 0) st->cnt[warp] = cnt;
             grp.sync();
             grp.finish(st, ckey, cidx, p.topk, p.part_idx + static_cast<size_t>(u) * p.topk,
@@ -418,15 +428,28 @@ cudaError_t launch_dec_t(const void* q, const float* q_scale, const void* k, con
     p.tiles_per_split = (nkt + p.splits - 1) / p.splits;
     p.splits = (nkt + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty units
     p.hdr = static_cast<WsHeader*>(ws);
+    unsigned char* scratch = static_cast<unsigned char*>(ws) + kWsHeaderBytes;
+    const bool radix = !paged;  // contiguous caches: score keys to memory, then the radix select
     const size_t parts = static_cast<size_t>(B) * p.splits * topk;
-    p.part_key = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + kWsHeaderBytes);
+    p.part_key = reinterpret_cast<uint32_t*>(scratch);
     p.part_idx = reinterpret_cast<int*>(p.part_key + parts);
+    p.score_keys = nullptr;
+    if (radix) {
+        p.part_key = nullptr;
+        p.part_idx = nullptr;
+        p.score_keys = reinterpret_cast<uint32_t*>(scratch);
+    }
     auto kern = indexer_decode_kernel<H, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     const int units = B * p.splits;
     kern<<<units < num_sms ? units : num_sms, C::THREADS, C::SMEM, stream>>>(mq, mk, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (radix) {
+        const size_t keys_bytes = (static_cast<size_t>(B) * max_len * 4 + 255) / 256 * 256;
+        return launch_radix_topk(p.score_keys, max_len, B, max_len, topk, idx_out, scratch + keys_bytes, num_sms,
+                                 stream);
+    }
     return launch_topk_merge_pairs(p.part_key, p.part_idx, B, p.splits * topk, topk, idx_out, p.hdr, num_sms,
                                    stream, max_len);
 }
@@ -442,6 +465,10 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
 }
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen) {
+    if (!varlen) {  // contiguous caches: the row's score keys, then the radix select's state
+        const size_t keys_bytes = (static_cast<size_t>(B) * (q_pos0 + 1) * 4 + 255) / 256 * 256;
+        return keys_bytes + radix_topk_scratch_bytes(B, q_pos0 + 1, num_sms);
+    }
     const int nkt = (q_pos0 + 1 + 127) / 128;  // varlen: q_pos0 = the longest sequence - 1
     int splits = dec_splits(B, nkt, num_sms, per_sm_for(B, varlen));
     const int tps = (nkt + splits - 1) / splits;

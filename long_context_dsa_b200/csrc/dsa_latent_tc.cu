@@ -93,6 +93,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 16 TMEM lanes (of this warp's quadrant) x 32 columns, twice: threads 0-15 read lanes 0-15 at
+// columns [col, col+32), threads 16-31 the same lanes at [col+32, col+64).  An M = 64 accumulator
+// keeps its rows in lanes 0-15 of each quadrant, so the whole warp shares one S row block.
+__device__ __forceinline__ void tmem_ld_16x32bx2(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+// Non-blocking: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // OR of `pred` over the `n` threads that meet at named barrier `id`.
 __device__ __forceinline__ bool bar_or(int id, int n, bool pred) {
     uint32_t r;
@@ -229,6 +257,15 @@ __global__ void __launch_bounds__(192, 1)
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             for (int j = 0; j < ntiles && ok; ++j, ++g) {
                 const int st = g & 1;
+                // lane: 4 keys (group kg) and half of the 9 column blocks; the index reads go out
+                // before the wait for the stage, so their latency hides behind it
+                const int kg = lane & 15;
+                int r[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int kk = j * NK + kg * 4 + i;
+                    r[i] = kk < p.topk ? __ldg(irow + kk) : -1;
+                }
                 if (lane == 0) {
                     if (g >= 2 && !mbar_wait(&kv_empty[st], ((g >> 1) - 1) & 1)) { fail(0x4c02); ok = false; }
                     if (ok && *abort_flag) ok = false;
@@ -236,13 +273,9 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                // lane: 4 keys (group kg) and half of the 9 column blocks
-                const int kg = lane & 15;
-                int r[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int kk = j * NK + kg * 4 + i;
-                    const int t = kk < p.topk ? __ldg(irow + kk) : -1;
+                    const int t = r[i];
                     if ((t < -1 || t >= p.n_kv) && lane < 16) raise_status(p.hdr, DSA_STATUS_BAD_INDEX, t);
                     const bool v = t >= 0 && t < p.n_kv && t <= lim;
                     r[i] = static_cast<int>(b * p.n_kv + (v ? t : 0));  // skipped entries read row 0 (masked)
@@ -264,56 +297,72 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::make_idesc(1, 1, 64, 64);
             constexpr uint32_t idesc_o = tc::make_idesc(1, 1, 128, 64) | (1u << 15);  // A (V^T) MN-major
-            uint32_t g = 0, sb = 0, pc = 0, uc = 0;
+            uint32_t g = 0, pc = 0, uc = 0;
             bool ok = true;
-            auto issue_s = [&](uint32_t gt, uint32_t sbt) -> bool {
-                const int st = gt & 1, bb = sbt & 1;
-                if (!mbar_wait(&kv_full[st], (gt >> 1) & 1)) return false;
-                if (sbt >= 2 && !mbar_wait(&s_empty[bb], ((sbt >> 1) - 1) & 1)) return false;
-                tc::fence_after_sync();
-                const uint32_t a0 = smem_u32(sQ), b0 = smem_u32(sSt + st * TILE);
-#pragma unroll 1
-                for (int c = 0; c < NBLK; ++c)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_f16(tmem + SCOL + bb * 64, sdesc(a0 + c * HB * 128 + kk * 32, 16, 1024),
-                                    sdesc(b0 + c * BLK + kk * 32, 16, 1024), idesc_s, (c | kk) != 0);
-                tc::mma_commit(&s_full[bb]);
-                return true;
-            };
+            // S(j+1) and PV(j) wait on different things (the gather of tile j+1, the softmax of tile
+            // j); the issuer polls both and issues whichever is ready, so a slow gather never holds
+            // back a PV that could free a stage for the next gather.
             for (long long u = blockIdx.x; u < units && ok; u += gridDim.x, ++uc) {
                 if (!mbar_wait(q_full, uc & 1)) { fail(0x4c11); break; }
-                const uint32_t g0 = g, sb0 = sb;
-                if (!issue_s(g0, sb0)) { fail(0x4c12); break; }
-                if (ntiles == 1) tc::mma_commit(q_empty);  // every S of this unit issued: Q may be refilled
-                for (int j = 0; j < ntiles; ++j) {
-                    if (j + 1 < ntiles) {
-                        if (!issue_s(g0 + j + 1, sb0 + j + 1)) { fail(0x4c13); ok = false; break; }
-                        if (j + 2 == ntiles) tc::mma_commit(q_empty);
-                    }
-                    // PV of tile j
-                    if (!mbar_wait(p_full, pc & 1)) { fail(0x4c14); ok = false; break; }
-                    ++pc;
-                    if (j == 0 && uc > 0 && !mbar_wait(o_free, (uc - 1) & 1)) { fail(0x4c15); ok = false; break; }
-                    tc::fence_after_sync();
-                    const int st = (g0 + j) & 1;
-                    const uint32_t v0 = smem_u32(sSt + st * TILE);
-                    const uint32_t phi = v0 + (NBLK - 1) * BLK, plo = smem_u32(sPlo);
+                const uint32_t g0 = g;
+                int ns = 0, np = 0;  // next S and next PV of this unit
+                uint64_t idle0 = 0;
+                while (np < ntiles) {
+                    bool prog = false;
+                    if (ns < ntiles && ns <= np + 1) {
+                        const uint32_t gt = g0 + ns;
+                        const int st = gt & 1, bb = gt & 1;
+                        if (mbar_test(&kv_full[st], (gt >> 1) & 1) &&
+                            (gt < 2 || mbar_test(&s_empty[bb], ((gt >> 1) - 1) & 1))) {
+                            tc::fence_after_sync();
+                            const uint32_t a0 = smem_u32(sQ), b0 = smem_u32(sSt + st * TILE);
 #pragma unroll 1
-                    for (int t = 0; t < 4; ++t)
+                            for (int c = 0; c < NBLK; ++c)
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            const uint64_t ad = sdesc(v0 + 2 * t * BLK + ks * 2048, BLK, 1024);
-                            const uint32_t d = tmem + OCOL + t * 64;
-                            tc::mma_f16(d, ad, sdesc(phi + ks * 32, 16, 1024), idesc_o, (j | ks) != 0);
-                            tc::mma_f16(d, ad, sdesc(plo + ks * 32, 16, 1024), idesc_o, true);
+                                for (int kk = 0; kk < 4; ++kk)
+                                    tc::mma_f16(tmem + SCOL + bb * 64, sdesc(a0 + c * HB * 128 + kk * 32, 16, 1024),
+                                                sdesc(b0 + c * BLK + kk * 32, 16, 1024), idesc_s, (c | kk) != 0);
+                            tc::mma_commit(&s_full[bb]);
+                            ++ns;
+                            if (ns == ntiles) tc::mma_commit(q_empty);  // every S of the unit issued
+                            prog = true;
                         }
-                    tc::mma_commit(&kv_empty[st]);
-                    tc::mma_commit(o_done);
-                    if (*abort_flag) { ok = false; break; }
+                    }
+                    if (np < ns && mbar_test(p_full, pc & 1) &&
+                        (np > 0 || uc == 0 || mbar_test(o_free, (uc - 1) & 1))) {
+                        ++pc;
+                        tc::fence_after_sync();
+                        const int st = (g0 + np) & 1;
+                        const uint32_t v0 = smem_u32(sSt + st * TILE);
+                        const uint32_t phi = v0 + (NBLK - 1) * BLK, plo = smem_u32(sPlo);
+#pragma unroll 1
+                        for (int t = 0; t < 4; ++t)
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) {
+                                const uint64_t ad = sdesc(v0 + 2 * t * BLK + ks * 2048, BLK, 1024);
+                                const uint32_t d = tmem + OCOL + t * 64;
+                                tc::mma_f16(d, ad, sdesc(phi + ks * 32, 16, 1024), idesc_o, (np | ks) != 0);
+                                tc::mma_f16(d, ad, sdesc(plo + ks * 32, 16, 1024), idesc_o, true);
+                            }
+                        tc::mma_commit(&kv_empty[st]);
+                        tc::mma_commit(o_done);
+                        ++np;
+                        prog = true;
+                    }
+                    if (prog) {
+                        idle0 = 0;
+                    } else {
+                        const uint64_t now = globaltimer_ns();
+                        if (idle0 == 0) {
+                            idle0 = now;
+                        } else if (now - idle0 > kWaitLimitNs || *abort_flag) {
+                            if (!*abort_flag) fail(0x4c14);
+                            ok = false;
+                            break;
+                        }
+                    }
                 }
                 g += ntiles;
-                sb += ntiles;
             }
             // nothing may still run on the tensor core when TMEM is released
             tc::mma_commit(drain);
@@ -321,9 +370,12 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ======================================================== softmax + epilogue (warps 0-3)
+        // Each head's S row (64 tokens) is shared by two lanes: lanes 0-15 take tokens 0-31 of heads
+        // 16q..16q+15, lanes 16-31 tokens 32-63 of the same heads (tcgen05.ld 16x32bx2).
         const int q = warp;                    // TMEM lane quadrant
-        const int h = 16 * q + lane;           // this thread's head (lanes 0-15 of the quadrant)
-        const bool own = lane < 16;
+        const int hl = lane & 15, half = lane >> 4;
+        const int h = 16 * q + hl;             // this thread's head
+        const bool lead = half == 0;           // writes the head's per-head values
         const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
         uint32_t sb = 0, oc = 0, uc = 0;
         bool ok = true;
@@ -333,7 +385,16 @@ __global__ void __launch_bounds__(192, 1)
             const int* irow;
             unit_row(u, row, hb, irow, lim, b);
             float m_run = -INFINITY, l_run = 0.f;
+            // entries of the current tile (lane i: entry i and 32 + i), read one tile ahead
+            int e0 = entry(irow, lim, lane), e1 = entry(irow, lim, 32 + lane);
             for (int j = 0; j < ntiles; ++j, ++sb) {
+                const uint32_t live0 = __ballot_sync(0xffffffffu, e0 >= 0);
+                const uint32_t live1 = __ballot_sync(0xffffffffu, e1 >= 0);
+                if (j + 1 < ntiles) {
+                    e0 = entry(irow, lim, (j + 1) * NK + lane);
+                    e1 = entry(irow, lim, (j + 1) * NK + 32 + lane);
+                }
+                const uint32_t live = half ? live1 : live0;  // this lane's 32 tokens
                 const int bb = sb & 1;
                 const bool got = mbar_wait(&s_full[bb], (sb >> 1) & 1);
                 if (bar_or(1, 128, !got)) {
@@ -342,22 +403,19 @@ __global__ void __launch_bounds__(192, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                uint32_t v[64];
-                tmem_ld64(tq + SCOL + bb * 64, v);
+                uint32_t v[32];
+                tmem_ld_16x32bx2(tq + SCOL + bb * 64, v);
+                tc::tmem_wait_ld_dep(v);
                 tc::fence_before_sync();
                 mbar_arrive(&s_empty[bb]);
-                // which of the tile's 64 entries are live
-                const int e0 = entry(irow, lim, j * NK + lane), e1 = entry(irow, lim, j * NK + 32 + lane);
-                const uint32_t live0 = __ballot_sync(0xffffffffu, e0 >= 0);
-                const uint32_t live1 = __ballot_sync(0xffffffffu, e1 >= 0);
                 float mx = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const bool lv = ((i < 32 ? live0 >> i : live1 >> (i - 32)) & 1u) != 0;
-                    const float s = lv ? __uint_as_float(v[i]) * p.scale_log2 : -INFINITY;
-                    v[i] = __float_as_uint(s);
-                    mx = fmaxf(mx, s);
+                for (int i = 0; i < 32; ++i) {
+                    const float sv = ((live >> i) & 1u) ? __uint_as_float(v[i]) * p.scale_log2 : -INFINITY;
+                    v[i] = __float_as_uint(sv);
+                    mx = fmaxf(mx, sv);
                 }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 const float m_new = fmaxf(m_run, mx);
                 bool resc = false;
                 float alpha = 1.f;
@@ -369,12 +427,13 @@ __global__ void __launch_bounds__(192, 1)
                     m_run = m_new;
                     l_run *= alpha;
                 }
-                const bool any = bar_or(2, 128, own && resc);
-                // P = 2^(s - m_run), as bf16 hi + lo; rows of P^T (64 tokens of head h) are 128 bytes
-                uint32_t hi[32], lo[32];
+                const bool any = bar_or(2, 128, resc);
+                // P = 2^(s - m_run), as bf16 hi + lo; a row of P^T (64 tokens of head h) is 128 bytes,
+                // this lane's half is its 16-byte chunks 4 half .. 4 half + 3
+                uint32_t hi[16], lo[16];
                 float lsum = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     const float s0 = __uint_as_float(v[2 * i]), s1 = __uint_as_float(v[2 * i + 1]);
                     const float p0 = (m_run == -INFINITY) ? 0.f : exp2f(s0 - m_run);
                     const float p1 = (m_run == -INFINITY) ? 0.f : exp2f(s1 - m_run);
@@ -383,16 +442,14 @@ __global__ void __launch_bounds__(192, 1)
                     const __nv_bfloat162 hh = *reinterpret_cast<const __nv_bfloat162*>(&hi[i]);
                     lo[i] = pack_bf16x2(p0 - __low2float(hh), p1 - __high2float(hh));
                 }
-                l_run += lsum;
+                l_run += lsum + __shfl_xor_sync(0xffffffffu, lsum, 16);
                 // P_hi goes to the rope block of this tile's stage: every role walks the same units and
                 // tiles, so the producer's and the MMA issuer's tile counter equals sb here
                 unsigned char* phi = sSt + (sb & 1) * TILE + (NBLK - 1) * BLK;
-                if (own) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(phi + sw128(h, c)) =
-                            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                }
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(phi + sw128(h, 4 * half + c)) =
+                        make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
                 if (j > 0) {
                     // PV of the previous tile done: P_lo may be rewritten, O^T is stable
                     const bool got2 = mbar_wait(o_done, oc & 1);
@@ -404,7 +461,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     tc::fence_after_sync();
                     if (any) {
-                        if (own) sAlpha[h] = resc ? alpha : 1.f;
+                        if (lead) sAlpha[h] = resc ? alpha : 1.f;
                         named_bar_sync(3, 128);
                         for (int t = 0; t < 4; ++t) {
                             uint32_t o[64];
@@ -418,12 +475,10 @@ __global__ void __launch_bounds__(192, 1)
                         named_bar_sync(3, 128);
                     }
                 }
-                if (own) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(sPlo + sw128(h, c)) =
-                            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-                }
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(sPlo + sw128(h, 4 * half + c)) =
+                        make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
                 fence_proxy_async_smem();  // P (generic writes) before the tensor core reads it
                 tc::fence_before_sync();
                 mbar_arrive(p_full);
@@ -437,7 +492,7 @@ __global__ void __launch_bounds__(192, 1)
                 break;
             }
             tc::fence_after_sync();
-            if (own) sL[h] = l_run > 0.f ? 1.f / l_run : 0.f;
+            if (lead) sL[h] = l_run > 0.f ? 1.f / l_run : 0.f;
             named_bar_sync(3, 128);
             const size_t obase = (static_cast<size_t>(row) * p.Hq + static_cast<size_t>(hb) * HB) * DV;
             for (int t = 0; t < 4; ++t) {

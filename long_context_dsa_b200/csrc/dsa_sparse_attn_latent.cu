@@ -271,18 +271,20 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 
 // Combine the split ranges of each (query row, head block): for every head,
 // O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s (a range that met only
-// skipped entries has m_s = -inf and drops out).  One block per unit, a warp per head at a
-// time; lane s holds range s's (m, l) (splits <= 32) and each lane owns DV/32 columns.
+// skipped entries has m_s = -inf and drops out).  One block per (unit, 4 heads), a warp per
+// head; lane s holds range s's (m, l) (splits <= 32) and each lane owns DV/32 columns.
 template <bool OUT_BF16>
-__global__ void __launch_bounds__(512)
+__global__ void __launch_bounds__(128)
     latent_merge_kernel(const float* __restrict__ part, int HB, int hblocks, int splits, int Hq,
                         void* __restrict__ O) {
-    const long long u = blockIdx.x;  // (row, head block)
+    const int hq4 = HB / 4;                     // blocks per unit
+    const long long u = blockIdx.x / hq4;       // (row, head block)
     const long long row = u / hblocks;
     const int hb = static_cast<int>(u % hblocks);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t sstride = static_cast<size_t>(HB) * (DV + 2);
-    for (int h = warp; h < HB; h += 16) {
+    {
+        const int h = static_cast<int>(blockIdx.x % hq4) * 4 + warp;
         const float* p0 = part + (static_cast<size_t>(u) * splits * HB + h) * (DV + 2);
         const float m = lane < splits ? __ldg(p0 + lane * sstride + DV) : -INFINITY;
         const float l = lane < splits ? __ldg(p0 + lane * sstride + DV + 1) : 0.f;
@@ -354,10 +356,11 @@ cudaError_t launch_w(const void* Q, const void* KV, const int* idx, int B, int n
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(KV), idx, B, n_q, n_kv, Hq, topk,
         scale * 1.4426950408889634f, O, splits, cps, part, share, hdr);
     if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    const unsigned mblocks = static_cast<unsigned>(units * (Cf::HB / 4));
     if (out_bf16)
-        latent_merge_kernel<true><<<static_cast<unsigned>(units), 512, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
+        latent_merge_kernel<true><<<mblocks, 128, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
     else
-        latent_merge_kernel<false><<<static_cast<unsigned>(units), 512, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
+        latent_merge_kernel<false><<<mblocks, 128, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
     return cudaGetLastError();
 }
 

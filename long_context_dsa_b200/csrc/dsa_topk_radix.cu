@@ -1,0 +1,252 @@
+// dsa_topk_radix.cu -- per-row top-k of a few long rows of score keys, spread over many CTAs.
+//
+// Same selection rule as every other top-k in the library ([Term] "dot product + top-k"; ties
+// to the lower token index, output ascending then -1): for a decode step the one-query indexer
+// writes its row of order-preserving score keys (4 bytes per cached token: 4 MB at a 1M-token
+// cache, against the 134 MB of fp8 keys it reads), and the selection runs here as a radix
+// select over all the row's keys, with every SM taking a slice:
+//   * 4 histogram passes of 8 bits each, from the top bit down.  Each CTA counts the keys of its
+//     slice that match the prefix found so far (shared-memory histogram, then global atomics);
+//     the last CTA of the row to finish (atomic ticket, no waiting) picks the digit holding the
+//     k-th key, extends the prefix and clears the histogram for the next pass.  After 4 passes
+//     the prefix is the k-th largest key K and `kk` says how many keys equal to K are selected.
+//   * A count pass: keys above K and keys equal to K in each slice.
+//   * A write pass: each CTA places its selected tokens (keys above K, and the first kk keys
+//     equal to K in token order) at their rank among the row's selections -- slices are token
+//     ranges in order, so the output is ascending -- and pads the row with -1.
+// No CTA ever waits for another: the passes are separate launches.
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kRxThreads = 256;
+
+struct RadixRow {
+    uint32_t prefix;  // the k-th key's bits found so far
+    int kk;           // how many of the keys matching the prefix are still to select
+    int ticket;       // CTAs of the row done with the current pass
+    int pad;
+};
+
+__global__ void __launch_bounds__(kRxThreads)
+    radix_init_kernel(RadixRow* rs, int* hist, int rows, int k) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * 256; i += gridDim.x * blockDim.x) hist[i] = 0;
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x) {
+        rs[r].prefix = 0u;
+        rs[r].kk = k;
+        rs[r].ticket = 0;
+        rs[r].pad = 0;
+    }
+}
+
+// Pass `pass` (0 = bits 31..24): histogram of the next 8 bits of the keys that match the prefix.
+__global__ void __launch_bounds__(kRxThreads)
+    radix_hist_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int pass, int k,
+                      RadixRow* rs, int* hist) {
+    __shared__ int sh[256];
+    __shared__ int last;
+    const int row = blockIdx.x / nblk, blk = blockIdx.x % nblk;
+    const int shift = 24 - 8 * pass;
+    const uint32_t fixed = pass == 0 ? 0u : (0xffffffffu << (32 - 8 * pass));
+    const uint32_t prefix = rs[row].prefix;
+    const int kk = rs[row].kk;
+    for (int b = threadIdx.x; b < 256; b += kRxThreads) sh[b] = 0;
+    __syncthreads();
+    if (n > k) {  // (rows no longer than k select everything; nothing to count)
+        const uint32_t* kr = keys + row * ld;
+        const int i0 = blk * per, i1 = min(n, i0 + per);
+        for (int i = i0 + threadIdx.x; i < i1; i += kRxThreads) {
+            const uint32_t key = __ldg(kr + i);
+            if ((key & fixed) == prefix) atomicAdd(&sh[(key >> shift) & 255u], 1);
+        }
+    }
+    __syncthreads();
+    int* hr = hist + row * 256;
+    for (int b = threadIdx.x; b < 256; b += kRxThreads)
+        if (sh[b]) atomicAdd(hr + b, sh[b]);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = (atomicAdd(&rs[row].ticket, 1) == nblk - 1);
+    __syncthreads();
+    if (!last) return;
+    // the row's last CTA: every other CTA's counts are in (they fenced before taking a ticket)
+    __threadfence();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int c8[8], s8 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            c8[j] = atomicAdd(hr + lane * 8 + j, 0);  // read through L2
+            s8 += c8[j];
+        }
+        int suf = s8;  // keys in bins >= lane*8
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_down_sync(0xffffffffu, suf, off);
+            if (lane + off < 32) suf += o;
+        }
+        const int need = min(kk, n);
+        const unsigned ball = __ballot_sync(0xffffffffu, suf >= need);
+        const int L = ball ? 31 - __clz(ball) : 0;
+        if (lane == L) {
+            int acc = suf - s8;
+            int d = 0, above = 0;
+            bool found = false;
+#pragma unroll
+            for (int j = 7; j >= 0; --j) {
+                if (!found && acc + c8[j] >= need) {
+                    d = L * 8 + j;
+                    above = acc;
+                    found = true;
+                }
+                acc += c8[j];
+            }
+            rs[row].prefix = prefix | (static_cast<uint32_t>(d) << shift);
+            rs[row].kk = need - above;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hr[lane * 8 + j] = 0;
+        if (lane == 0) rs[row].ticket = 0;
+    }
+}
+
+// Keys above the k-th key and keys equal to it, per slice.
+__global__ void __launch_bounds__(kRxThreads)
+    radix_count_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int k,
+                       const RadixRow* rs, int2* counts) {
+    __shared__ int wg[kRxThreads / 32], we[kRxThreads / 32];
+    const int row = blockIdx.x / nblk, blk = blockIdx.x % nblk;
+    const uint32_t K = rs[row].prefix;
+    const uint32_t* kr = keys + row * ld;
+    const int i0 = blk * per, i1 = min(n, i0 + per);
+    int g = 0, e = 0;
+    if (n > k)
+        for (int i = i0 + threadIdx.x; i < i1; i += kRxThreads) {
+            const uint32_t key = __ldg(kr + i);
+            g += key > K;
+            e += key == K;
+        }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, off);
+        e += __shfl_xor_sync(0xffffffffu, e, off);
+    }
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        wg[w] = g;
+        we[w] = e;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int tg = 0, te = 0;
+        for (int j = 0; j < kRxThreads / 32; ++j) {
+            tg += wg[j];
+            te += we[j];
+        }
+        counts[blockIdx.x] = make_int2(tg, te);
+    }
+}
+
+// Selected tokens of each slice, at their rank among the row's selections; -1 after the last.
+__global__ void __launch_bounds__(kRxThreads)
+    radix_write_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int k,
+                       const RadixRow* rs, const int2* counts, int* __restrict__ out) {
+    __shared__ int wsel[kRxThreads / 32], weq[kRxThreads / 32];
+    __shared__ int base_out, base_eq;
+    const int row = blockIdx.x / nblk, blk = blockIdx.x % nblk;
+    int* orow = out + static_cast<long long>(row) * k;
+    const int i0 = blk * per, i1 = min(n, i0 + per);
+    if (n <= k) {  // every token of the row, then padding
+        for (int i = i0 + threadIdx.x; i < i1; i += kRxThreads) orow[i] = i;
+        if (blk == nblk - 1)
+            for (int j = n + threadIdx.x; j < k; j += kRxThreads) orow[j] = -1;
+        return;
+    }
+    const uint32_t K = rs[row].prefix;
+    const int kk = rs[row].kk;  // keys equal to K to take, lowest tokens first
+    if (threadIdx.x == 0) {
+        int o = 0, eb = 0;
+        for (int j = 0; j < blk; ++j) {
+            const int2 c = counts[row * nblk + j];
+            o += c.x + min(max(kk - eb, 0), c.y);
+            eb += c.y;
+        }
+        base_out = o;
+        base_eq = eb;
+    }
+    __syncthreads();
+    int o = base_out, eb = base_eq;
+    const uint32_t* kr = keys + row * ld;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int c0 = i0; c0 < i1; c0 += kRxThreads) {
+        const int i = c0 + threadIdx.x;
+        const uint32_t key = i < i1 ? __ldg(kr + i) : 0u;
+        const bool eq = i < i1 && key == K;
+        const bool gt = i < i1 && key > K;
+        // rank of this equal key among the row's equal keys, in token order
+        const unsigned meq = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) weq[w] = __popc(meq);
+        __syncthreads();
+        int eq_before = eb;
+        for (int j = 0; j < w; ++j) eq_before += weq[j];
+        eq_before += __popc(meq & ((1u << lane) - 1u));
+        const bool sel = gt || (eq && eq_before < kk);
+        const unsigned msel = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) wsel[w] = __popc(msel);
+        __syncthreads();
+        int pos = o;
+        for (int j = 0; j < w; ++j) pos += wsel[j];
+        pos += __popc(msel & ((1u << lane) - 1u));
+        if (sel && pos < k) orow[pos] = i;
+        int tsel = 0, teq = 0;
+        for (int j = 0; j < kRxThreads / 32; ++j) {
+            tsel += wsel[j];
+            teq += weq[j];
+        }
+        o += tsel;
+        eb += teq;
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+// Slices per row: enough CTAs to cover the SMs about four times, slices of at least 4096 keys.
+int radix_blocks(int rows, int n, int num_sms, int* per) {
+    int nblk = (4 * num_sms + rows - 1) / rows;
+    const int most = (n + 4095) / 4096;
+    if (nblk > most) nblk = most;
+    if (nblk < 1) nblk = 1;
+    *per = (n + nblk - 1) / nblk;
+    *per = (*per + kRxThreads - 1) / kRxThreads * kRxThreads;
+    nblk = (n + *per - 1) / *per;
+    return nblk < 1 ? 1 : nblk;
+}
+
+size_t radix_topk_scratch_bytes(int rows, int n, int num_sms) {
+    int per = 0;
+    const int nblk = radix_blocks(rows, n, num_sms, &per);
+    return static_cast<size_t>(rows) * (sizeof(RadixRow) + 256 * sizeof(int)) +
+           static_cast<size_t>(rows) * nblk * sizeof(int2);
+}
+
+// Top-k of `rows` rows of n keys (row stride ld) -> out [rows, k] ascending tokens, then -1.
+cudaError_t launch_radix_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
+                              int num_sms, cudaStream_t stream) {
+    int per = 0;
+    const int nblk = radix_blocks(rows, n, num_sms, &per);
+    RadixRow* rs = static_cast<RadixRow*>(scratch);
+    int* hist = reinterpret_cast<int*>(rs + rows);
+    int2* counts = reinterpret_cast<int2*>(hist + static_cast<size_t>(rows) * 256);
+    const unsigned grid = static_cast<unsigned>(rows) * nblk;
+    radix_init_kernel<<<(rows * 256 + kRxThreads - 1) / kRxThreads, kRxThreads, 0, stream>>>(rs, hist, rows, k);
+    for (int pass = 0; pass < 4; ++pass)
+        radix_hist_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, pass, k, rs, hist);
+    radix_count_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, rs, counts);
+    radix_write_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, rs, counts, out);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -124,9 +124,9 @@ def test_indexer_survivors_concentrated_in_one_lane_range():
     assert frac > 0.9
 
 
-def test_decode_long_cache_uses_streaming_merge():
-    """A 1.7M-token cache: the position bitmap of the split merge would not fit in shared memory,
-    so the streaming merge of the partial lists runs; the selection is still the oracle's."""
+def test_decode_long_cache():
+    """One query against a 1.7M-token cache (the score keys of the row, then the multi-CTA radix
+    select); the selection follows the oracle's rule."""
     B, L, H, d, k = 1, 1_700_000, 32, 128, 2048
     g = synth.StructuredIndexer("long_decode", B, L, H, d, r=32, base_std=1.0, noise_std=0.2, seed=0)
     kk = g.keys(0)

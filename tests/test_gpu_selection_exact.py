@@ -7,7 +7,8 @@ index, ascending output, -1 padding) leaves exactly one correct answer.  Small v
 ranges make equal scores and zero scores common, so tie-breaking, the streaming prune of
 the fused kernel (and its exact fallback when one score value holds more ties than the
 prune's slack), the split decode kernel's partial lists and both of its merges are all
-checked for exactness, not within a tolerance.
+checked for exactness, not within a tolerance; so is the multi-CTA radix select that one-query
+decode over a contiguous cache uses.
 
 [QbitAI] §IndexCache / [Term] "dot product + top-k": the selection is the k best scores
 of each query row; ties to the lower index is this library's stated rule.
@@ -140,10 +141,30 @@ def test_decode_fp8_selection_is_exact():
     _decode_case("dec_fp8_b3", 3, 12000, 64, 2048, -3, 3, fp8=True)
 
 
-def test_decode_streaming_merge_selection_is_exact():
-    """A 1.7M-token cache: the position bitmap would not fit in shared memory, so the split
-    lists go through the streaming merge."""
-    _decode_case("dec_stream", 1, 1_700_000, 32, 2048, -2, 2)
+def test_decode_long_cache_selection_is_exact():
+    """One query against a 1.7M-token cache: the score keys of the whole row go through the
+    multi-CTA radix select."""
+    _decode_case("dec_long", 1, 1_700_000, 32, 2048, -2, 2)
+
+
+def test_paged_decode_streaming_merge_selection_is_exact():
+    """A paged sequence of 1.7M tokens: the position bitmap of the split merge would not fit in
+    shared memory, so the split lists go through the streaming merge."""
+    n, P, H, d, topk = 1_700_000, 256, 32, 128, 2048
+    q, k, w = synth.integer_indexer("paged_stream", 1, n, H, d, -2, 2, q_rows=1)
+    pages = (n + P - 1) // P
+    perm = np.random.default_rng(5).permutation(pages).astype(np.int32)
+    pool = torch.zeros((pages * P, d), dtype=torch.bfloat16)
+    pool.view(pages, P, d)[torch.from_numpy(perm).long()] = torch.cat(
+        [k[0], torch.zeros((pages * P - n, d), dtype=torch.bfloat16)]).view(pages, P, d)
+    table = torch.from_numpy(perm[None]).to(DEV)
+    ws = torch.zeros(dsa.idx_score_topk_paged_workspace_size(1, n, H, d, topk), dtype=torch.uint8, device=DEV)
+    idx = dsa.idx_score_topk_paged(q[:, 0].contiguous().to(DEV), pool.view(pages, P, d).to(DEV), table,
+                                   torch.tensor([n], dtype=torch.int32, device=DEV), w[:, 0].contiguous().to(DEV),
+                                   topk, n, workspace=ws)
+    assert dsa.read_status(ws) == 0
+    sc = oracle.indexer_scores(q[0], k[0], w[0], n - 1)
+    _expect_identical(idx.cpu().numpy(), oracle.topk_select(sc, topk, n - 1), "paged 1.7M")
 
 
 def test_paged_decode_selection_is_exact():
