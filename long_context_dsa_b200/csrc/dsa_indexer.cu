@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(320, 1)
         TopkRowState* st = sSt + g * C::QG;
         int* sortbuf = sSort + g * DSA_TOPK_MAX;
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + g * 256;
-        constexpr int CHECK = 4;                       // prune checks every CHECK key tiles
+        constexpr int CHECK = 8;                       // prune checks every CHECK key tiles
         const int sub = grp.sub();                     // this warp's share of a row buffer
         const int room = sub - CHECK * 32;             // prune once a sub-buffer holds more than this
         const int slack = max(32, p.topk / 8);         // a prune may keep up to k + slack candidates
@@ -362,8 +362,8 @@ __global__ void __launch_bounds__(320, 1)
                             const bool valid = full_tile | ((q < qlast) & (s_key <= pos0 + q));
                             // admit iff the score ranks above the row's k-th candidate (set by the last prune)
                             const uint32_t key = score_key(sc[q]);
-                            const uint32_t tk = st[q].thr_key;
-                            const bool adm = valid & ((key > tk) | ((key == tk) & (s_key < st[q].thr_idx)));
+                            const uint2 th = *reinterpret_cast<const uint2*>(&st[q].thr_key);  // (key, idx)
+                            const bool adm = valid & ((key > th.x) | ((key == th.x) & (s_key < static_cast<int>(th.y))));
                             topk_append_warp(wkey + q * rstride, widx + q * rstride, cnt[q], key, s_key, adm, sub);
                         }
                     }

@@ -29,6 +29,8 @@
 #include "dsa_tc.cuh"
 
 namespace dsa {
+cudaError_t launch_latent_merge(const float* part, int HB, int hblocks, int splits, long long units, int Hq, void* O,
+                                bool out_bf16, cudaStream_t stream);
 namespace lattc {
 
 constexpr int DQK = 576, DV = 512, HB = 64, NK = 64;
@@ -148,6 +150,8 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) {
 struct Params {
     const int* idx;
     int B, n_q, n_kv, Hq, topk, hblocks;
+    int splits, tps;  // each unit's tiles in `splits` ranges of `tps` tiles (1 range: no split)
+    float* part;      // splits > 1: per (item, head) unnormalised O^T, max and sum; merged afterwards
     float scale_log2;
     void* O;
     IdxShare share;
@@ -181,7 +185,14 @@ __global__ void __launch_bounds__(192, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long units = static_cast<long long>(p.B) * p.n_q * p.hblocks;
+    const long long items = units * p.splits;
     const int ntiles = (p.topk + NK - 1) / NK;
+    // item -> (unit, first tile, tiles): a unit's tiles are cut into ranges when units are few
+    auto item_tiles = [&](long long it, long long& u, int& t0, int& nt) {
+        u = it / p.splits;
+        t0 = static_cast<int>(it % p.splits) * p.tps;
+        nt = min(ntiles, t0 + p.tps) - t0;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -239,10 +250,11 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t g = 0, uc = 0;
         int q_issued = -1;  // last unit whose query block was requested (lane 0)
         bool ok = true;
-        for (long long u = blockIdx.x; u < units && ok; u += gridDim.x, ++uc) {
-            long long row, b;
-            int hb, lim;
+        for (long long it = blockIdx.x; it < items && ok; it += gridDim.x, ++uc) {
+            long long u, row, b;
+            int hb, lim, t0, nt;
             const int* irow;
+            item_tiles(it, u, t0, nt);
             unit_row(u, row, hb, irow, lim, b);
             if (lane == 0) {
                 if (uc > 0 && !mbar_wait(q_empty, (uc - 1) & 1)) { fail(0x4c01); ok = false; }
@@ -255,7 +267,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            for (int j = 0; j < ntiles && ok; ++j, ++g) {
+            for (int j = 0; j < nt && ok; ++j, ++g) {
                 const int st = g & 1;
                 // lane: 4 keys (group kg) and half of the 9 column blocks; the index reads go out
                 // before the wait for the stage, so their latency hides behind it
@@ -263,7 +275,7 @@ __global__ void __launch_bounds__(192, 1)
                 int r[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int kk = j * NK + kg * 4 + i;
+                    const int kk = (t0 + j) * NK + kg * 4 + i;
                     r[i] = kk < p.topk ? __ldg(irow + kk) : -1;
                 }
                 if (lane == 0) {
@@ -302,14 +314,17 @@ __global__ void __launch_bounds__(192, 1)
             // S(j+1) and PV(j) wait on different things (the gather of tile j+1, the softmax of tile
             // j); the issuer polls both and issues whichever is ready, so a slow gather never holds
             // back a PV that could free a stage for the next gather.
-            for (long long u = blockIdx.x; u < units && ok; u += gridDim.x, ++uc) {
+            for (long long it = blockIdx.x; it < items && ok; it += gridDim.x, ++uc) {
+                long long u;
+                int t0, nt;
+                item_tiles(it, u, t0, nt);
                 if (!mbar_wait(q_full, uc & 1)) { fail(0x4c11); break; }
                 const uint32_t g0 = g;
-                int ns = 0, np = 0;  // next S and next PV of this unit
+                int ns = 0, np = 0;  // next S and next PV of this item
                 uint64_t idle0 = 0;
-                while (np < ntiles) {
+                while (np < nt) {
                     bool prog = false;
-                    if (ns < ntiles && ns <= np + 1) {
+                    if (ns < nt && ns <= np + 1) {
                         const uint32_t gt = g0 + ns;
                         const int st = gt & 1, bb = gt & 1;
                         if (mbar_test(&kv_full[st], (gt >> 1) & 1) &&
@@ -324,7 +339,7 @@ __global__ void __launch_bounds__(192, 1)
                                                 sdesc(b0 + c * BLK + kk * 32, 16, 1024), idesc_s, (c | kk) != 0);
                             tc::mma_commit(&s_full[bb]);
                             ++ns;
-                            if (ns == ntiles) tc::mma_commit(q_empty);  // every S of the unit issued
+                            if (ns == nt) tc::mma_commit(q_empty);  // every S of the item issued
                             prog = true;
                         }
                     }
@@ -362,7 +377,7 @@ __global__ void __launch_bounds__(192, 1)
                         }
                     }
                 }
-                g += ntiles;
+                g += nt;
             }
             // nothing may still run on the tensor core when TMEM is released
             tc::mma_commit(drain);
@@ -379,20 +394,21 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
         uint32_t sb = 0, oc = 0, uc = 0;
         bool ok = true;
-        for (long long u = blockIdx.x; u < units && ok; u += gridDim.x, ++uc) {
-            long long row, b;
-            int hb, lim;
+        for (long long it = blockIdx.x; it < items && ok; it += gridDim.x, ++uc) {
+            long long u, row, b;
+            int hb, lim, t0, nt;
             const int* irow;
+            item_tiles(it, u, t0, nt);
             unit_row(u, row, hb, irow, lim, b);
             float m_run = -INFINITY, l_run = 0.f;
             // entries of the current tile (lane i: entry i and 32 + i), read one tile ahead
-            int e0 = entry(irow, lim, lane), e1 = entry(irow, lim, 32 + lane);
-            for (int j = 0; j < ntiles; ++j, ++sb) {
+            int e0 = entry(irow, lim, t0 * NK + lane), e1 = entry(irow, lim, t0 * NK + 32 + lane);
+            for (int j = 0; j < nt; ++j, ++sb) {
                 const uint32_t live0 = __ballot_sync(0xffffffffu, e0 >= 0);
                 const uint32_t live1 = __ballot_sync(0xffffffffu, e1 >= 0);
-                if (j + 1 < ntiles) {
-                    e0 = entry(irow, lim, (j + 1) * NK + lane);
-                    e1 = entry(irow, lim, (j + 1) * NK + 32 + lane);
+                if (j + 1 < nt) {
+                    e0 = entry(irow, lim, (t0 + j + 1) * NK + lane);
+                    e1 = entry(irow, lim, (t0 + j + 1) * NK + 32 + lane);
                 }
                 const uint32_t live = half ? live1 : live0;  // this lane's 32 tokens
                 const int bb = sb & 1;
@@ -492,6 +508,25 @@ __global__ void __launch_bounds__(192, 1)
                 break;
             }
             tc::fence_after_sync();
+            if (p.part) {
+                // a range of the unit's tiles: unnormalised O^T and (max, sum) per head, [item][head][DV + 2]
+                float* pb = p.part + static_cast<size_t>(it) * HB * (DV + 2);
+                if (lead) {
+                    pb[static_cast<size_t>(h) * (DV + 2) + DV] = m_run;
+                    pb[static_cast<size_t>(h) * (DV + 2) + DV + 1] = l_run;
+                }
+                for (int t = 0; t < 4; ++t) {
+                    uint32_t o[64];
+                    tmem_ld64(tq + OCOL + t * 64, o);
+                    const int d = t * 128 + q * 32 + lane;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) pb[static_cast<size_t>(i) * (DV + 2) + d] = __uint_as_float(o[i]);
+                }
+                tc::fence_before_sync();
+                named_bar_sync(3, 128);
+                mbar_arrive(o_free);
+                continue;
+            }
             if (lead) sL[h] = l_run > 0.f ? 1.f / l_run : 0.f;
             named_bar_sync(3, 128);
             const size_t obase = (static_cast<size_t>(row) * p.Hq + static_cast<size_t>(hb) * HB) * DV;
@@ -550,15 +585,14 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows
 
 }  // namespace lattc
 
-// The tensor-core form serves query heads in blocks of 64 when there are at least as many
-// (row, head block) units as SMs; smaller problems take the split warp-MMA kernel.
-bool latent_tc_applies(int B, int n_q, int Hq, int num_sms) {
-    return Hq % lattc::HB == 0 && static_cast<long long>(B) * n_q * (Hq / lattc::HB) >= num_sms;
-}
+// The tensor-core form serves query heads in blocks of 64.  With fewer (row, head block) units
+// than SMs (decode) each unit's tiles are cut into ranges, at most `max_splits` (the warp-MMA
+// kernel's split count for the same shape, which sizes the workspace), merged afterwards.
+bool latent_tc_applies(int Hq) { return Hq % lattc::HB == 0; }
 
 cudaError_t launch_latent_tc(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv, int Hq,
                              int topk, float scale, void* O, bool out_bf16, IdxShare share, WsHeader* hdr,
-                             int num_sms, cudaStream_t stream) {
+                             int max_splits, int num_sms, cudaStream_t stream) {
     using namespace lattc;
     CUtensorMap mq, mkv;
     if (!make_map(&mq, Q, static_cast<uint64_t>(B) * n_q * Hq, HB) ||
@@ -576,13 +610,25 @@ cudaError_t launch_latent_tc(const void* Q, const void* KV, const int* idx, int 
     p.O = O;
     p.share = share;
     p.hdr = hdr;
+    const long long units = static_cast<long long>(B) * n_q * p.hblocks;
+    const int ntiles = (topk + NK - 1) / NK;
+    int splits = 1;
+    if (units < num_sms && max_splits > 1) {
+        splits = static_cast<int>((num_sms + units - 1) / units);
+        if (splits > max_splits) splits = max_splits;
+        if (splits > ntiles) splits = ntiles;
+    }
+    p.tps = (ntiles + splits - 1) / splits;
+    p.splits = (ntiles + p.tps - 1) / p.tps;
+    p.part = p.splits > 1 ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(hdr) + kWsHeaderBytes) : nullptr;
     auto kern = out_bf16 ? latent_tc_kernel<true> : latent_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
-    const long long units = static_cast<long long>(B) * n_q * p.hblocks;
-    const int grid = units < num_sms ? static_cast<int>(units) : num_sms;
+    const long long items = units * p.splits;
+    const int grid = items < num_sms ? static_cast<int>(items) : num_sms;
     kern<<<grid, 192, SMEM, stream>>>(mq, mkv, p);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess || p.splits == 1) return e;
+    return launch_latent_merge(p.part, HB, p.hblocks, p.splits, units, Hq, O, out_bf16, stream);
 }
 
 }  // namespace dsa

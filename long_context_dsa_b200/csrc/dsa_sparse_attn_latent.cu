@@ -271,21 +271,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 
 // Combine the split ranges of each (query row, head block): for every head,
 // O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s (a range that met only
-// skipped entries has m_s = -inf and drops out).  One block per (unit, 4 heads), a warp per
-// head; lane s holds range s's (m, l) (splits <= 32) and each lane owns DV/32 columns.
+// skipped entries has m_s = -inf and drops out).  One 128-thread block per (unit, head): the
+// first warp turns the ranges' (m, l) into weights in shared memory (splits <= 32), then each
+// thread accumulates 4 of the 512 output columns over the ranges.
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(128)
     latent_merge_kernel(const float* __restrict__ part, int HB, int hblocks, int splits, int Hq,
                         void* __restrict__ O) {
-    const int hq4 = HB / 4;                     // blocks per unit
-    const long long u = blockIdx.x / hq4;       // (row, head block)
+    __shared__ float wt[32];
+    __shared__ float inv_l;
+    const long long u = blockIdx.x / HB;  // (row, head block)
+    const int h = static_cast<int>(blockIdx.x % HB);
     const long long row = u / hblocks;
     const int hb = static_cast<int>(u % hblocks);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t sstride = static_cast<size_t>(HB) * (DV + 2);
-    {
-        const int h = static_cast<int>(blockIdx.x % hq4) * 4 + warp;
-        const float* p0 = part + (static_cast<size_t>(u) * splits * HB + h) * (DV + 2);
+    const float* p0 = part + (static_cast<size_t>(u) * splits * HB + h) * (DV + 2);
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
         const float m = lane < splits ? __ldg(p0 + lane * sstride + DV) : -INFINITY;
         const float l = lane < splits ? __ldg(p0 + lane * sstride + DV + 1) : 0.f;
         float M = m;
@@ -295,25 +297,49 @@ __global__ void __launch_bounds__(128)
         float L = f * l;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        float acc[DV / 32];
-#pragma unroll
-        for (int i = 0; i < DV / 32; ++i) acc[i] = 0.f;
-        for (int s2 = 0; s2 < splits; ++s2) {
-            const float fs = __shfl_sync(0xffffffffu, f, s2);
-#pragma unroll
-            for (int i = 0; i < DV / 32; ++i) acc[i] += fs * __ldg(p0 + s2 * sstride + i * 32 + lane);
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const size_t ob = (static_cast<size_t>(row) * Hq + static_cast<size_t>(hb) * HB + h) * DV;
-#pragma unroll
-        for (int i = 0; i < DV / 32; ++i) {
-            if (OUT_BF16)
-                reinterpret_cast<__nv_bfloat16*>(O)[ob + i * 32 + lane] = __float2bfloat16_rn(acc[i] * inv);
-            else
-                reinterpret_cast<float*>(O)[ob + i * 32 + lane] = acc[i] * inv;
-        }
+        wt[lane] = f;
+        if (lane == 0) inv_l = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    const int d = threadIdx.x * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int s2 = 0; s2 < splits; ++s2) {
+        const float fs = wt[s2];
+        const float* src = p0 + s2 * sstride + d;
+        // rows of DV + 2 floats: 8-byte aligned, so two float2 loads
+        const float2 a = __ldg(reinterpret_cast<const float2*>(src));
+        const float2 c = __ldg(reinterpret_cast<const float2*>(src + 2));
+        acc.x += fs * a.x;
+        acc.y += fs * a.y;
+        acc.z += fs * c.x;
+        acc.w += fs * c.y;
+    }
+    const float inv = inv_l;
+    const size_t ob = (static_cast<size_t>(row) * Hq + static_cast<size_t>(hb) * HB + h) * DV + d;
+    if (OUT_BF16) {
+        __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(O) + ob;
+        *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        *reinterpret_cast<__nv_bfloat162*>(op + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    } else {
+        float* op = reinterpret_cast<float*>(O) + ob;
+        *reinterpret_cast<float4*>(op) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
 }
+
+}  // namespace lat
+
+cudaError_t launch_latent_merge(const float* part, int HB, int hblocks, int splits, long long units, int Hq, void* O,
+                                bool out_bf16, cudaStream_t stream) {
+    const unsigned mblocks = static_cast<unsigned>(units * HB);
+    if (out_bf16)
+        lat::latent_merge_kernel<true><<<mblocks, 128, 0, stream>>>(part, HB, hblocks, splits, Hq, O);
+    else
+        lat::latent_merge_kernel<false><<<mblocks, 128, 0, stream>>>(part, HB, hblocks, splits, Hq, O);
+    return cudaGetLastError();
+}
+
+namespace lat {
 
 // Warps per CTA (8 query heads each) for Hq query heads.
 inline int warps_for(int Hq) { return Hq % 64 == 0 ? 8 : Hq % 32 == 0 ? 4 : Hq % 16 == 0 ? 2 : 1; }
@@ -356,20 +382,15 @@ cudaError_t launch_w(const void* Q, const void* KV, const int* idx, int B, int n
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(KV), idx, B, n_q, n_kv, Hq, topk,
         scale * 1.4426950408889634f, O, splits, cps, part, share, hdr);
     if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
-    const unsigned mblocks = static_cast<unsigned>(units * (Cf::HB / 4));
-    if (out_bf16)
-        latent_merge_kernel<true><<<mblocks, 128, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
-    else
-        latent_merge_kernel<false><<<mblocks, 128, 0, stream>>>(part, Cf::HB, hblocks, splits, Hq, O);
-    return cudaGetLastError();
+    return launch_latent_merge(part, Cf::HB, hblocks, splits, units, Hq, O, out_bf16, stream);
 }
 
 }  // namespace lat
 
-bool latent_tc_applies(int B, int n_q, int Hq, int num_sms);
+bool latent_tc_applies(int Hq);
 cudaError_t launch_latent_tc(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv, int Hq,
                              int topk, float scale, void* O, bool out_bf16, IdxShare share, WsHeader* hdr,
-                             int num_sms, cudaStream_t stream);
+                             int max_splits, int num_sms, cudaStream_t stream);
 
 // Many query rows with heads in blocks of 64: the tensor-core kernel (dsa_latent_tc.cu).  Otherwise
 // (decode, a few rows, other head counts) the warp-MMA kernel above, with split ranges when the
@@ -377,8 +398,13 @@ cudaError_t launch_latent_tc(const void* Q, const void* KV, const int* idx, int 
 cudaError_t launch_sparse_attn_latent(const void* Q, const void* KV, const int* idx, int B, int n_q, int n_kv,
                                       int Hq, int topk, float scale, void* O, bool out_bf16, IdxShare share,
                                       WsHeader* hdr, int num_sms, cudaStream_t stream) {
-    if (latent_tc_applies(B, n_q, Hq, num_sms))
-        return launch_latent_tc(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
+    if (latent_tc_applies(Hq)) {
+        const long long units = static_cast<long long>(B) * n_q * (Hq / 64);
+        int cps = 0;
+        const int max_splits = lat::latent_splits(units, (topk + lat::CHUNK - 1) / lat::CHUNK, num_sms, &cps);
+        return launch_latent_tc(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, max_splits,
+                                num_sms, stream);
+    }
     switch (lat::warps_for(Hq)) {
         case 8: return lat::launch_w<8>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);
         case 4: return lat::launch_w<4>(Q, KV, idx, B, n_q, n_kv, Hq, topk, scale, O, out_bf16, share, hdr, num_sms, stream);

@@ -57,9 +57,18 @@ __global__ void __launch_bounds__(kRxThreads)
     if (n > k) {  // (rows no longer than k select everything; nothing to count)
         const uint32_t* kr = keys + row * ld;
         const int i0 = blk * per, i1 = min(n, i0 + per);
-        for (int i = i0 + threadIdx.x; i < i1; i += kRxThreads) {
-            const uint32_t key = __ldg(kr + i);
-            if ((key & fixed) == prefix) atomicAdd(&sh[(key >> shift) & 255u], 1);
+        // the keys of a row share their top bits, so most lanes of a warp hit the same bin:
+        // one shared-memory atomic per distinct digit per warp
+        for (int c0 = i0; c0 < i1; c0 += kRxThreads) {
+            const int i = c0 + threadIdx.x;
+            const uint32_t key = i < i1 ? __ldg(kr + i) : 0u;
+            const bool in = i < i1 && (key & fixed) == prefix;
+            const unsigned active = __ballot_sync(0xffffffffu, in);
+            if (in) {
+                const uint32_t dg = (key >> shift) & 255u;
+                const unsigned same = __match_any_sync(active, dg);
+                if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sh[dg], __popc(same));
+            }
         }
     }
     __syncthreads();
@@ -166,17 +175,35 @@ __global__ void __launch_bounds__(kRxThreads)
     }
     const uint32_t K = rs[row].prefix;
     const int kk = rs[row].kk;  // keys equal to K to take, lowest tokens first
-    if (threadIdx.x == 0) {
-        int o = 0, eb = 0;
-        for (int j = 0; j < blk; ++j) {
+    {
+        // keys above K and keys equal to K in the slices before this one (the block sums them)
+        int g = 0, e = 0;
+        for (int j = threadIdx.x; j < blk; j += kRxThreads) {
             const int2 c = counts[row * nblk + j];
-            o += c.x + min(max(kk - eb, 0), c.y);
-            eb += c.y;
+            g += c.x;
+            e += c.y;
         }
-        base_out = o;
-        base_eq = eb;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, off);
+            e += __shfl_xor_sync(0xffffffffu, e, off);
+        }
+        if ((threadIdx.x & 31) == 0) {
+            wsel[threadIdx.x >> 5] = g;
+            weq[threadIdx.x >> 5] = e;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int tg = 0, te = 0;
+            for (int j = 0; j < kRxThreads / 32; ++j) {
+                tg += wsel[j];
+                te += weq[j];
+            }
+            base_out = tg + min(te, kk);  // equal keys are taken in token order
+            base_eq = te;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     int o = base_out, eb = base_eq;
     const uint32_t* kr = keys + row * ld;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
