@@ -742,6 +742,8 @@ def run_decode(args, dev):
         att_ms = sum(evs[3 * l + 1].elapsed_time(evs[3 * l + 2]) for l in range(4))
         res[p] = (ms, idx_ms, att_ms)
     ms, idx_ms, att_ms = res[pat]
+    graph_ms = decode_graph_ms(lambda: [dsa.layer_group_forward(shape, layers, pat, cache, workspace=ws)
+                                        for _ in range(10)], 10, ws)
     kbytes = B * Lc * D_I * 2  # the key cache one F layer scans
     abytes = B * TOPK * HKV * 2 * DH * 2
     del layers
@@ -749,6 +751,7 @@ def run_decode(args, dev):
     return {"workload": f"decode B={B} at a {Lc}-token cache, 4 layers {pat}, H_I={H_I} d_I={D_I} top-{TOPK}, "
                         f"GQA {HQ}Q/{HKV}KV d={DH}",
             "tok_per_s": round(B / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+            "graph_tok_per_s": _finite(B / (graph_ms / 1e3), 1), "graph_ms_per_step": _finite(graph_ms, 4),
             "indexer_ms": round(idx_ms, 4), "attention_ms": round(att_ms, 4),
             "indexer_gbs": round(kbytes / (idx_ms / 1e3) / 1e9, 1),
             "attention_gathered_gbs": round(4 * abytes / (att_ms / 1e3) / 1e9, 1),
@@ -1159,6 +1162,46 @@ def _ctx1m_caches(dev, n_kv, n_layers=N_LAYERS, seed=3000):
     return gen, keys, lat
 
 
+def _finite(x, nd):
+    """x rounded to nd places, or None when it is not a finite number."""
+    import math
+    return round(x, nd) if math.isfinite(x) else None
+
+
+def decode_graph_ms(run_steps, steps, ws, reps=5):
+    """Capture `run_steps` (issues `steps` decode steps through the library on the current stream)
+    into one CUDA graph, replay it and return ms per step (CUDA events around the replays)."""
+    import torch
+    from long_context_dsa_b200 import dsa
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run_steps()  # warm every launch path on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            run_steps()
+    except Exception as e:  # reported, not fatal: the eager numbers stand on their own
+        torch.cuda.synchronize()
+        print(f"decode graph capture failed: {e}", file=sys.stderr)
+        return float("nan")
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    dsa.check_status(ws)
+    ms = a.elapsed_time(b) / (reps * steps)
+    del g
+    return ms
+
+
 def run_decode1m(args, dev):
     """Decode after the 1M-token prefill: 32 steps, batch 1, the new token at positions 1048576 ..
     1048607 (the cache grows from 1048577 to 1048608 tokens); 8 layers FSSSFSSS, fp8 indexer H_I=64
@@ -1214,6 +1257,9 @@ def run_decode1m(args, dev):
     ms = a.elapsed_time(b) / steps
     idx_ms = sum(es[3 * l].elapsed_time(es[3 * l + 1]) for es in evs for l in range(N_LAYERS)) / steps
     att_ms = sum(es[3 * l + 1].elapsed_time(es[3 * l + 2]) for es in evs for l in range(N_LAYERS)) / steps
+    # the same 32 steps captured once into a CUDA graph and replayed: at batch 1 a step is ~20 small
+    # launches, so the host's launch rate matters; the graph removes it
+    graph_ms = decode_graph_ms(lambda: [step(s) for s in range(steps)], steps, ws)
     hbm = peaks()[0]
     n_f = PATTERN.count("F")
     kbytes = n_f * (L1 + steps // 2) * (D_I + 4)            # fp8 keys + fp32 scales per F layer
@@ -1225,8 +1271,10 @@ def run_decode1m(args, dev):
                         f"indexer H_I={H1} d_I={D_I} top-{TOPK}, latent attention 576/512 with {HQ1} heads",
             "tok_per_s": round(1e3 / ms, 1), "ms_per_step": round(ms, 4),
             "indexer_ms_per_step": round(idx_ms, 4), "attention_ms_per_step": round(att_ms, 4),
+            "graph_tok_per_s": _finite(1e3 / graph_ms, 1), "graph_ms_per_step": _finite(graph_ms, 4),
             "hbm_bound_ms_per_step": round(bound_s * 1e3, 4),
             "frac_of_hbm_bound": round(bound_s * 1e3 / ms, 4),
+            "graph_frac_of_hbm_bound": _finite(bound_s * 1e3 / graph_ms, 4),
             "bound_note": "fp8 keys + scales of the 2 F layers and 2048 latent rows of each of 8 layers, read "
                           "once at measured HBM bandwidth"}
 

@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* o_done = bars + 11;
     uint64_t* o_free = bars + 12;
     uint64_t* drain = bars + 13;
+    uint64_t* plo_free = bars + 14;  // the P_lo half of a PV is done: P_lo may be rewritten
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(p_full, 128);
         mbar_init(o_done, 1);
+        mbar_init(plo_free, 1);
         mbar_init(o_free, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -350,15 +352,21 @@ __global__ void __launch_bounds__(192, 1)
                         const int st = (g0 + np) & 1;
                         const uint32_t v0 = smem_u32(sSt + st * TILE);
                         const uint32_t phi = v0 + (NBLK - 1) * BLK, plo = smem_u32(sPlo);
+                        // the P_lo products first, so the softmax may refill P_lo while the P_hi
+                        // products still run
 #pragma unroll 1
                         for (int t = 0; t < 4; ++t)
 #pragma unroll
-                            for (int ks = 0; ks < 4; ++ks) {
-                                const uint64_t ad = sdesc(v0 + 2 * t * BLK + ks * 2048, BLK, 1024);
-                                const uint32_t d = tmem + OCOL + t * 64;
-                                tc::mma_f16(d, ad, sdesc(phi + ks * 32, 16, 1024), idesc_o, (np | ks) != 0);
-                                tc::mma_f16(d, ad, sdesc(plo + ks * 32, 16, 1024), idesc_o, true);
-                            }
+                            for (int ks = 0; ks < 4; ++ks)
+                                tc::mma_f16(tmem + OCOL + t * 64, sdesc(v0 + 2 * t * BLK + ks * 2048, BLK, 1024),
+                                            sdesc(plo + ks * 32, 16, 1024), idesc_o, (np | ks) != 0);
+                        tc::mma_commit(plo_free);
+#pragma unroll 1
+                        for (int t = 0; t < 4; ++t)
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                tc::mma_f16(tmem + OCOL + t * 64, sdesc(v0 + 2 * t * BLK + ks * 2048, BLK, 1024),
+                                            sdesc(phi + ks * 32, 16, 1024), idesc_o, true);
                         tc::mma_commit(&kv_empty[st]);
                         tc::mma_commit(o_done);
                         ++np;
@@ -367,6 +375,7 @@ __global__ void __launch_bounds__(192, 1)
                     if (prog) {
                         idle0 = 0;
                     } else {
+                        __nanosleep(32);  // leave the issue slots to the softmax warp sharing this sub-partition
                         const uint64_t now = globaltimer_ns();
                         if (idle0 == 0) {
                             idle0 = now;
@@ -393,7 +402,7 @@ __global__ void __launch_bounds__(192, 1)
         const bool lead = half == 0;           // writes the head's per-head values
         const uint32_t tq = tmem + (static_cast<uint32_t>(q * 32) << 16);
         uint32_t sb = 0, oc = 0, uc = 0;
-        bool ok = true;
+        bool ok = true, pv_waited = false;
         for (long long it = blockIdx.x; it < items && ok; it += gridDim.x, ++uc) {
             long long u, row, b;
             int hb, lim, t0, nt;
@@ -467,9 +476,13 @@ __global__ void __launch_bounds__(192, 1)
                     *reinterpret_cast<uint4*>(phi + sw128(h, 4 * half + c)) =
                         make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
                 if (j > 0) {
-                    // PV of the previous tile done: P_lo may be rewritten, O^T is stable
-                    const bool got2 = mbar_wait(o_done, oc & 1);
-                    ++oc;
+                    // the previous tile's PV has read P_lo (its P_lo products come first); with a
+                    // rescale the whole PV must be done, so that O^T is stable
+                    bool got2 = mbar_wait(plo_free, (oc - 1) & 1);
+                    if (got2 && any) {
+                        got2 = mbar_wait(o_done, (oc - 1) & 1);
+                        pv_waited = true;
+                    }
                     if (bar_or(1, 128, !got2)) {
                         if (lane == 0 && !got2) fail(0x4c22);
                         ok = false;
@@ -498,11 +511,21 @@ __global__ void __launch_bounds__(192, 1)
                 fence_proxy_async_smem();  // P (generic writes) before the tensor core reads it
                 tc::fence_before_sync();
                 mbar_arrive(p_full);
+                if (j > 0 && !pv_waited) {
+                    // consume the previous PV's completion in order (its products are done by now)
+                    const bool got3 = mbar_wait(o_done, (oc - 1) & 1);
+                    if (bar_or(1, 128, !got3)) {
+                        if (lane == 0 && !got3) fail(0x4c24);
+                        ok = false;
+                        break;
+                    }
+                }
+                pv_waited = false;
+                ++oc;  // oc: PVs issued so far, this tile's included
             }
             if (!ok) break;
             // ---- epilogue: O = O^T / l, written row-major [head][d]
-            const bool got = mbar_wait(o_done, oc & 1);
-            ++oc;
+            const bool got = mbar_wait(o_done, (oc - 1) & 1);
             if (bar_or(1, 128, !got)) {
                 if (lane == 0 && !got) fail(0x4c23);
                 break;

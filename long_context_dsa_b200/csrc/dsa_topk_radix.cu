@@ -5,10 +5,10 @@
 // writes its row of order-preserving score keys (4 bytes per cached token: 4 MB at a 1M-token
 // cache, against the 134 MB of fp8 keys it reads), and the selection runs here as a radix
 // select over all the row's keys, with every SM taking a slice:
-//   * 4 histogram passes of 8 bits each, from the top bit down.  Each CTA counts the keys of its
+//   * 3 histogram passes of 11, 11 and 10 bits, from the top bit down.  Each CTA counts the keys of its
 //     slice that match the prefix found so far (shared-memory histogram, then global atomics);
 //     the last CTA of the row to finish (atomic ticket, no waiting) picks the digit holding the
-//     k-th key, extends the prefix and clears the histogram for the next pass.  After 4 passes
+//     k-th key, extends the prefix and clears the histogram for the next pass.  After 3 passes
 //     the prefix is the k-th largest key K and `kk` says how many keys equal to K are selected.
 //   * A count pass: keys above K and keys equal to K in each slice.
 //   * A write pass: each CTA places its selected tokens (keys above K, and the first kk keys
@@ -22,6 +22,10 @@ namespace dsa {
 namespace {
 
 constexpr int kRxThreads = 256;
+constexpr int kRxBins = 2048;  // 11-bit digits
+// pass p covers bits [shift, shift + width) of the key
+__host__ __device__ constexpr int rx_shift(int pass) { return pass == 0 ? 21 : pass == 1 ? 10 : 0; }
+__host__ __device__ constexpr int rx_width(int pass) { return pass == 2 ? 10 : 11; }
 
 struct RadixRow {
     uint32_t prefix;  // the k-th key's bits found so far
@@ -32,7 +36,7 @@ struct RadixRow {
 
 __global__ void __launch_bounds__(kRxThreads)
     radix_init_kernel(RadixRow* rs, int* hist, int rows, int k) {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * 256; i += gridDim.x * blockDim.x) hist[i] = 0;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows * kRxBins; i += gridDim.x * blockDim.x) hist[i] = 0;
     for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x) {
         rs[r].prefix = 0u;
         rs[r].kk = k;
@@ -41,18 +45,19 @@ __global__ void __launch_bounds__(kRxThreads)
     }
 }
 
-// Pass `pass` (0 = bits 31..24): histogram of the next 8 bits of the keys that match the prefix.
+// Pass `pass` (0 = bits 31..21): histogram of the next digit of the keys that match the prefix.
 __global__ void __launch_bounds__(kRxThreads)
     radix_hist_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int pass, int k,
                       RadixRow* rs, int* hist) {
-    __shared__ int sh[256];
+    __shared__ int sh[kRxBins];
     __shared__ int last;
     const int row = blockIdx.x / nblk, blk = blockIdx.x % nblk;
-    const int shift = 24 - 8 * pass;
-    const uint32_t fixed = pass == 0 ? 0u : (0xffffffffu << (32 - 8 * pass));
+    const int shift = rx_shift(pass);
+    const uint32_t dmask = (1u << rx_width(pass)) - 1u;
+    const uint32_t fixed = pass == 0 ? 0u : (0xffffffffu << (shift + rx_width(pass)));
     const uint32_t prefix = rs[row].prefix;
     const int kk = rs[row].kk;
-    for (int b = threadIdx.x; b < 256; b += kRxThreads) sh[b] = 0;
+    for (int b = threadIdx.x; b < kRxBins; b += kRxThreads) sh[b] = 0;
     __syncthreads();
     if (n > k) {  // (rows no longer than k select everything; nothing to count)
         const uint32_t* kr = keys + row * ld;
@@ -65,15 +70,15 @@ __global__ void __launch_bounds__(kRxThreads)
             const bool in = i < i1 && (key & fixed) == prefix;
             const unsigned active = __ballot_sync(0xffffffffu, in);
             if (in) {
-                const uint32_t dg = (key >> shift) & 255u;
+                const uint32_t dg = (key >> shift) & dmask;
                 const unsigned same = __match_any_sync(active, dg);
                 if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sh[dg], __popc(same));
             }
         }
     }
     __syncthreads();
-    int* hr = hist + row * 256;
-    for (int b = threadIdx.x; b < 256; b += kRxThreads)
+    int* hr = hist + row * kRxBins;
+    for (int b = threadIdx.x; b < kRxBins; b += kRxThreads)
         if (sh[b]) atomicAdd(hr + b, sh[b]);
     __threadfence();
     __syncthreads();
@@ -83,14 +88,12 @@ __global__ void __launch_bounds__(kRxThreads)
     // the row's last CTA: every other CTA's counts are in (they fenced before taking a ticket)
     __threadfence();
     if (threadIdx.x < 32) {
+        // lane l owns bins 64 l .. 64 l + 63; the digit holding the need-th largest key
         const int lane = threadIdx.x;
-        int c8[8], s8 = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            c8[j] = atomicAdd(hr + lane * 8 + j, 0);  // read through L2
-            s8 += c8[j];
-        }
-        int suf = s8;  // keys in bins >= lane*8
+        constexpr int PB = kRxBins / 32;
+        int s64 = 0;
+        for (int j = 0; j < PB; ++j) s64 += atomicAdd(hr + lane * PB + j, 0);  // read through L2
+        int suf = s64;  // keys in bins >= lane * PB
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_down_sync(0xffffffffu, suf, off);
@@ -100,23 +103,22 @@ __global__ void __launch_bounds__(kRxThreads)
         const unsigned ball = __ballot_sync(0xffffffffu, suf >= need);
         const int L = ball ? 31 - __clz(ball) : 0;
         if (lane == L) {
-            int acc = suf - s8;
+            int acc = suf - s64;
             int d = 0, above = 0;
-            bool found = false;
-#pragma unroll
-            for (int j = 7; j >= 0; --j) {
-                if (!found && acc + c8[j] >= need) {
-                    d = L * 8 + j;
+            for (int j = PB - 1; j >= 0; --j) {
+                const int c = atomicAdd(hr + lane * PB + j, 0);
+                if (acc + c >= need) {
+                    d = lane * PB + j;
                     above = acc;
-                    found = true;
+                    break;
                 }
-                acc += c8[j];
+                acc += c;
             }
             rs[row].prefix = prefix | (static_cast<uint32_t>(d) << shift);
             rs[row].kk = need - above;
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) hr[lane * 8 + j] = 0;
+        __syncwarp();
+        for (int j = 0; j < PB; ++j) hr[lane * PB + j] = 0;
         if (lane == 0) rs[row].ticket = 0;
     }
 }
@@ -255,7 +257,7 @@ int radix_blocks(int rows, int n, int num_sms, int* per) {
 size_t radix_topk_scratch_bytes(int rows, int n, int num_sms) {
     int per = 0;
     const int nblk = radix_blocks(rows, n, num_sms, &per);
-    return static_cast<size_t>(rows) * (sizeof(RadixRow) + 256 * sizeof(int)) +
+    return static_cast<size_t>(rows) * (sizeof(RadixRow) + kRxBins * sizeof(int)) +
            static_cast<size_t>(rows) * nblk * sizeof(int2);
 }
 
@@ -266,10 +268,10 @@ cudaError_t launch_radix_topk(const uint32_t* keys, long long ld, int rows, int 
     const int nblk = radix_blocks(rows, n, num_sms, &per);
     RadixRow* rs = static_cast<RadixRow*>(scratch);
     int* hist = reinterpret_cast<int*>(rs + rows);
-    int2* counts = reinterpret_cast<int2*>(hist + static_cast<size_t>(rows) * 256);
+    int2* counts = reinterpret_cast<int2*>(hist + static_cast<size_t>(rows) * kRxBins);
     const unsigned grid = static_cast<unsigned>(rows) * nblk;
-    radix_init_kernel<<<(rows * 256 + kRxThreads - 1) / kRxThreads, kRxThreads, 0, stream>>>(rs, hist, rows, k);
-    for (int pass = 0; pass < 4; ++pass)
+    radix_init_kernel<<<(rows * kRxBins + kRxThreads - 1) / kRxThreads, kRxThreads, 0, stream>>>(rs, hist, rows, k);
+    for (int pass = 0; pass < 3; ++pass)
         radix_hist_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, pass, k, rs, hist);
     radix_count_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, rs, counts);
     radix_write_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, rs, counts, out);
