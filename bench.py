@@ -693,6 +693,36 @@ def run_profile_latent(args):
     print(json.dumps({"case": "profile_latent", "ms": t, "gathered_gbs": by / t / 1e6, "tflops": fl / t / 1e9}))
 
 
+def run_profile_decode1m(args):
+    """One-query fp8 decode indexer at a 1048577-token cache (H_I=64, d_I=128, top-2048) for ncu
+    captures: the split decode kernel writing the row's score keys, then the radix select."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    dev = torch.device("cuda", 0)
+    n = (1 << 20) + 1
+    gen = synth.StructuredIndexer("profdec1m", 1, n, 64, D_I, r=32, base_std=1.0, noise_std=SIGMA_1M, device=dev,
+                                  seed=9)
+    q, w = gen.queries(0, n - 1, n)
+    k8, ks = synth.quantize_e4m3_rows(gen.keys(0))
+    q8, qs = synth.quantize_e4m3_rows(q)
+    del gen
+    ws = torch.zeros(dsa.idx_score_topk_workspace_size(1, 1, n - 1, n, 64, D_I, TOPK, dsa.DSA_E4M3),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((1, 1, TOPK), dtype=torch.int32, device=dev)
+    ts = []
+    for it in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dsa.idx_score_topk(q8, k8, w, TOPK, q_pos0=n - 1, q_scale=qs, k_scale=ks, out=out, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    dsa.check_status(ws)
+    print(json.dumps({"case": "profile_decode1m", "ms": min(ts), "key_gbs": n * (D_I + 4) / min(ts) / 1e6}))
+
+
 def run_decode(args, dev):
     """Decode step: 64 sequences, one new token each, at a 200000-token cache; 4 layers FSSS
     (H_I=32, d_I=128, top-2048; attention 32 query / 4 KV heads, d=128)."""
@@ -1433,7 +1463,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench",
                     choices=["bench", "profile", "profile_paged", "decode", "decode_mha", "ctx1m", "mtp", "paged",
-                             "prefill16k", "decode1m", "ctx1m_full", "profile_latent", "cp"],
+                             "prefill16k", "decode1m", "ctx1m_full", "profile_latent", "profile_decode1m", "cp"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m / ...: only "
                          "that extra measurement, printed as one JSON line; cp: one 200K sequence split over "
                          "the torchrun ranks (context-parallel prefill, strong scaling)")
@@ -1446,6 +1476,9 @@ def main():
         return
     if args.case == "profile_latent":
         run_profile_latent(args)
+        return
+    if args.case == "profile_decode1m":
+        run_profile_decode1m(args)
         return
     extra_cases = {"decode": run_decode, "decode_mha": run_decode_mha, "ctx1m": run_ctx1m, "mtp": run_mtp,
                    "paged": run_paged, "prefill16k": run_prefill16k, "decode1m": run_decode1m,

@@ -286,6 +286,10 @@ __global__ void __launch_bounds__(320, 1)
             const int pos0 = p.q_pos0 + qg0;
 
             for (int j = 0; j < nkt; ++j, ++u) {
+                // fp8: this key's scale, read before the wait so its latency hides behind it
+                const int s_key0 = j * 128 + tid;
+                const float ksc = (FP8 && s_key0 < p.n_kv) ? __ldg(p.k_scale + static_cast<size_t>(b) * p.n_kv + s_key0)
+                                                            : 0.f;
                 const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[g], u & 1));
                 if (!got) {
                     if (lane == 0) {
@@ -342,7 +346,6 @@ __global__ void __launch_bounds__(320, 1)
 
                     const int s_key = j * 128 + tid;  // key position within the batch
                     if (FP8) {
-                        const float ksc = (s_key < p.n_kv) ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s_key] : 0.f;
 #pragma unroll
                         for (int q = 0; q < C::QG; ++q) sc[q] *= ksc;
                     }

@@ -269,6 +269,9 @@ __global__ void __launch_bounds__(192, 1)
             int* widx = cidx + warp * sub;
             for (int j = j0; j < j1; ++j, ++ua) {
                 const int a = ua % C::NACC;
+                const int s_key = j * 128 + tid;
+                // fp8: this key's scale, read before the wait so its latency hides behind it
+                const float ksc = (FP8 && s_key < len) ? __ldg(p.k_scale + static_cast<size_t>(b) * p.n_kv + s_key) : 0.f;
                 const bool got = __all_sync(0xffffffffu, mbar_wait(&acc_full[a], (ua / C::NACC) & 1));
                 float sc_v = 0.f;
                 if (got) {
@@ -296,8 +299,7 @@ __global__ void __launch_bounds__(192, 1)
                     atomicExch(abort_flag, 1);
                     *wg_abort = 1;
                 }
-                const int s_key = j * 128 + tid;
-                if (FP8) sc_v *= (s_key < len) ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s_key] : 0.f;
+                if (FP8) sc_v *= ksc;
                 const uint32_t key = score_key(sc_v);
                 if (p.score_keys) {
                     // score mode: the row's keys go to memory and a multi-CTA radix select picks the top-k

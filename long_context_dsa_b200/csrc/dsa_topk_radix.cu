@@ -5,10 +5,10 @@
 // writes its row of order-preserving score keys (4 bytes per cached token: 4 MB at a 1M-token
 // cache, against the 134 MB of fp8 keys it reads), and the selection runs here as a radix
 // select over all the row's keys, with every SM taking a slice:
-//   * 3 histogram passes of 11, 11 and 10 bits, from the top bit down.  Each CTA counts the keys of its
+//   * 4 histogram passes of 8 bits each, from the top bit down.  Each CTA counts the keys of its
 //     slice that match the prefix found so far (shared-memory histogram, then global atomics);
 //     the last CTA of the row to finish (atomic ticket, no waiting) picks the digit holding the
-//     k-th key, extends the prefix and clears the histogram for the next pass.  After 3 passes
+//     k-th key, extends the prefix and clears the histogram for the next pass.  After 4 passes
 //     the prefix is the k-th largest key K and `kk` says how many keys equal to K are selected.
 //   * A count pass: keys above K and keys equal to K in each slice.
 //   * A write pass: each CTA places its selected tokens (keys above K, and the first kk keys
@@ -22,10 +22,12 @@ namespace dsa {
 namespace {
 
 constexpr int kRxThreads = 256;
-constexpr int kRxBins = 2048;  // 11-bit digits
-// pass p covers bits [shift, shift + width) of the key
-__host__ __device__ constexpr int rx_shift(int pass) { return pass == 0 ? 21 : pass == 1 ? 10 : 0; }
-__host__ __device__ constexpr int rx_width(int pass) { return pass == 2 ? 10 : 11; }
+constexpr int kRxBins = 256;  // 8-bit digits (wider digits cost more in histogram clears and
+                               // flushes than the pass they save: measured with 3 x 11 bits)
+constexpr int kRxPasses = 4;
+// pass p covers bits [shift, shift + 8) of the key
+__host__ __device__ constexpr int rx_shift(int pass) { return 24 - 8 * pass; }
+__host__ __device__ constexpr int rx_width(int pass) { return 8 + 0 * pass; }
 
 struct RadixRow {
     uint32_t prefix;  // the k-th key's bits found so far
@@ -45,7 +47,7 @@ __global__ void __launch_bounds__(kRxThreads)
     }
 }
 
-// Pass `pass` (0 = bits 31..21): histogram of the next digit of the keys that match the prefix.
+// Pass `pass` (0 = bits 31..24): histogram of the next digit of the keys that match the prefix.
 __global__ void __launch_bounds__(kRxThreads)
     radix_hist_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int pass, int k,
                       RadixRow* rs, int* hist) {
@@ -63,16 +65,26 @@ __global__ void __launch_bounds__(kRxThreads)
         const uint32_t* kr = keys + row * ld;
         const int i0 = blk * per, i1 = min(n, i0 + per);
         // the keys of a row share their top bits, so most lanes of a warp hit the same bin:
-        // one shared-memory atomic per distinct digit per warp
-        for (int c0 = i0; c0 < i1; c0 += kRxThreads) {
-            const int i = c0 + threadIdx.x;
-            const uint32_t key = i < i1 ? __ldg(kr + i) : 0u;
-            const bool in = i < i1 && (key & fixed) == prefix;
-            const unsigned active = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const uint32_t dg = (key >> shift) & dmask;
-                const unsigned same = __match_any_sync(active, dg);
-                if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sh[dg], __popc(same));
+        // one shared-memory atomic per distinct digit per warp.  Keys are read kBatch at a time
+        // into registers first, so the loads overlap instead of waiting behind each vote.
+        constexpr int kBatch = 8;
+        for (int c0 = i0; c0 < i1; c0 += kRxThreads * kBatch) {
+            uint32_t kv[kBatch];
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) {
+                const int i = c0 + e * kRxThreads + threadIdx.x;
+                kv[e] = i < i1 ? __ldg(kr + i) : 0u;
+            }
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) {
+                const int i = c0 + e * kRxThreads + threadIdx.x;
+                const bool in = i < i1 && (kv[e] & fixed) == prefix;
+                const unsigned active = __ballot_sync(0xffffffffu, in);
+                if (in) {
+                    const uint32_t dg = (kv[e] >> shift) & dmask;
+                    const unsigned same = __match_any_sync(active, dg);
+                    if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sh[dg], __popc(same));
+                }
             }
         }
     }
@@ -88,7 +100,7 @@ __global__ void __launch_bounds__(kRxThreads)
     // the row's last CTA: every other CTA's counts are in (they fenced before taking a ticket)
     __threadfence();
     if (threadIdx.x < 32) {
-        // lane l owns bins 64 l .. 64 l + 63; the digit holding the need-th largest key
+        // lane l owns bins 8 l .. 8 l + 7; the digit holding the need-th largest key
         const int lane = threadIdx.x;
         constexpr int PB = kRxBins / 32;
         int s64 = 0;
@@ -161,10 +173,42 @@ __global__ void __launch_bounds__(kRxThreads)
 }
 
 // Selected tokens of each slice, at their rank among the row's selections; -1 after the last.
+// Each thread takes a contiguous run of the slice: it counts its keys above K and equal to K, one
+// block-wide scan gives every thread its rank among the equal keys and among the selections,
+// then the thread writes its selected tokens in order.
+__device__ __forceinline__ int2 block_excl_scan2(int2 v, int2* warp_tot, int2* total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int2 inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int ox = __shfl_up_sync(0xffffffffu, inc.x, off), oy = __shfl_up_sync(0xffffffffu, inc.y, off);
+        if (lane >= off) {
+            inc.x += ox;
+            inc.y += oy;
+        }
+    }
+    if (lane == 31) warp_tot[w] = inc;
+    __syncthreads();
+    int2 before = make_int2(0, 0), tot = make_int2(0, 0);
+#pragma unroll
+    for (int j = 0; j < kRxThreads / 32; ++j) {
+        const int2 t = warp_tot[j];
+        if (j < w) {
+            before.x += t.x;
+            before.y += t.y;
+        }
+        tot.x += t.x;
+        tot.y += t.y;
+    }
+    __syncthreads();
+    *total = tot;
+    return make_int2(before.x + inc.x - v.x, before.y + inc.y - v.y);
+}
+
 __global__ void __launch_bounds__(kRxThreads)
     radix_write_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int k,
                        const RadixRow* rs, const int2* counts, int* __restrict__ out) {
-    __shared__ int wsel[kRxThreads / 32], weq[kRxThreads / 32];
+    __shared__ int2 wt[kRxThreads / 32];
     __shared__ int base_out, base_eq;
     const int row = blockIdx.x / nblk, blk = blockIdx.x % nblk;
     int* orow = out + static_cast<long long>(row) * k;
@@ -178,65 +222,48 @@ __global__ void __launch_bounds__(kRxThreads)
     const uint32_t K = rs[row].prefix;
     const int kk = rs[row].kk;  // keys equal to K to take, lowest tokens first
     {
-        // keys above K and keys equal to K in the slices before this one (the block sums them)
-        int g = 0, e = 0;
+        // keys above K and keys equal to K in the slices before this one
+        int2 c = make_int2(0, 0);
         for (int j = threadIdx.x; j < blk; j += kRxThreads) {
-            const int2 c = counts[row * nblk + j];
-            g += c.x;
-            e += c.y;
+            const int2 x = counts[row * nblk + j];
+            c.x += x.x;
+            c.y += x.y;
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            g += __shfl_xor_sync(0xffffffffu, g, off);
-            e += __shfl_xor_sync(0xffffffffu, e, off);
-        }
-        if ((threadIdx.x & 31) == 0) {
-            wsel[threadIdx.x >> 5] = g;
-            weq[threadIdx.x >> 5] = e;
-        }
-        __syncthreads();
+        int2 tot;
+        block_excl_scan2(c, wt, &tot);
         if (threadIdx.x == 0) {
-            int tg = 0, te = 0;
-            for (int j = 0; j < kRxThreads / 32; ++j) {
-                tg += wsel[j];
-                te += weq[j];
-            }
-            base_out = tg + min(te, kk);  // equal keys are taken in token order
-            base_eq = te;
+            base_out = tot.x + min(tot.y, kk);  // equal keys are taken in token order
+            base_eq = tot.y;
         }
         __syncthreads();
     }
-    int o = base_out, eb = base_eq;
     const uint32_t* kr = keys + row * ld;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    for (int c0 = i0; c0 < i1; c0 += kRxThreads) {
-        const int i = c0 + threadIdx.x;
-        const uint32_t key = i < i1 ? __ldg(kr + i) : 0u;
-        const bool eq = i < i1 && key == K;
-        const bool gt = i < i1 && key > K;
-        // rank of this equal key among the row's equal keys, in token order
-        const unsigned meq = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) weq[w] = __popc(meq);
-        __syncthreads();
-        int eq_before = eb;
-        for (int j = 0; j < w; ++j) eq_before += weq[j];
-        eq_before += __popc(meq & ((1u << lane) - 1u));
-        const bool sel = gt || (eq && eq_before < kk);
-        const unsigned msel = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) wsel[w] = __popc(msel);
-        __syncthreads();
-        int pos = o;
-        for (int j = 0; j < w; ++j) pos += wsel[j];
-        pos += __popc(msel & ((1u << lane) - 1u));
-        if (sel && pos < k) orow[pos] = i;
-        int tsel = 0, teq = 0;
-        for (int j = 0; j < kRxThreads / 32; ++j) {
-            tsel += wsel[j];
-            teq += weq[j];
+    const int ipt = (per + kRxThreads - 1) / kRxThreads;  // this thread's run: [a, b)
+    const int a = min(i1, i0 + threadIdx.x * ipt), b = min(i1, a + ipt);
+    int2 mine = make_int2(0, 0);  // (above K, equal to K) in the run
+    for (int i = a; i < b; ++i) {
+        const uint32_t key = __ldg(kr + i);
+        mine.x += key > K;
+        mine.y += key == K;
+    }
+    int2 tot;
+    const int2 pre = block_excl_scan2(mine, wt, &tot);  // within the slice
+    int eq_rank = base_eq + pre.y;                        // equal keys before this run, row-wide
+    // selections before this run: keys above K, plus the equal keys that made the cut
+    int2 sel_mine = make_int2(mine.x + min(max(kk - eq_rank, 0), mine.y), 0);
+    int2 tsel;
+    int pos = base_out + block_excl_scan2(sel_mine, wt, &tsel).x;
+    for (int i = a; i < b; ++i) {
+        const uint32_t key = __ldg(kr + i);
+        bool sel = key > K;
+        if (key == K) {
+            sel = eq_rank < kk;
+            ++eq_rank;
         }
-        o += tsel;
-        eb += teq;
-        __syncthreads();
+        if (sel) {
+            if (pos < k) orow[pos] = i;
+            ++pos;
+        }
     }
 }
 
@@ -271,7 +298,7 @@ cudaError_t launch_radix_topk(const uint32_t* keys, long long ld, int rows, int 
     int2* counts = reinterpret_cast<int2*>(hist + static_cast<size_t>(rows) * kRxBins);
     const unsigned grid = static_cast<unsigned>(rows) * nblk;
     radix_init_kernel<<<(rows * kRxBins + kRxThreads - 1) / kRxThreads, kRxThreads, 0, stream>>>(rs, hist, rows, k);
-    for (int pass = 0; pass < 3; ++pass)
+    for (int pass = 0; pass < kRxPasses; ++pass)
         radix_hist_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, pass, k, rs, hist);
     radix_count_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, rs, counts);
     radix_write_kernel<<<grid, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, rs, counts, out);
