@@ -138,10 +138,14 @@ __global__ void __launch_bounds__(WARPS * 32)
         const __nv_bfloat16* vb = V + seq_off + static_cast<size_t>(g) * D;
         const int n_valid = PAGED ? min(__ldg(pg.lens + b), pg.max_pages * pg.page_size) : n_kv;
 
-        // cache row of key `lane` of chunk c (-1 past the end); out-of-range entries are flagged and skipped
-        auto load_idx = [&](int c) -> int {
+        // Index of key `lane` of chunk c (-1 past the end), read two chunks ahead of its gather, then
+        // checked and mapped to its cache row one chunk ahead (so a page-table read never waits on
+        // the index read it depends on); out-of-range entries are flagged and skipped.
+        auto load_raw = [&](int c) -> int {
             const int kk = c * CHUNK + lane;
-            int t = (lane < CHUNK && kk < topk) ? __ldg(irow + kk) : -1;
+            return (lane < CHUNK && kk < topk) ? __ldg(irow + kk) : -1;
+        };
+        auto map_idx = [&](int t) -> int {
             if (t < -1 || t >= n_valid) {
                 raise_status(hdr, DSA_STATUS_BAD_INDEX, t);
                 t = -1;
@@ -194,15 +198,18 @@ __global__ void __launch_bounds__(WARPS * 32)
         for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
         float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
 
-        // prologue: stages 0 .. STAGES-2 in flight, the next chunk's indices in a register
+        // prologue: stages 0 .. STAGES-2 in flight, the next chunk's rows and the one after's
+        // indices in registers
         __syncwarp();
 #pragma unroll
-        for (int c = 0; c < STAGES - 1; ++c) issue(c0 + c, load_idx(c0 + c));
-        int t_next = load_idx(c0 + STAGES - 1);
+        for (int c = 0; c < STAGES - 1; ++c) issue(c0 + c, map_idx(load_raw(c0 + c)));
+        int t_next = map_idx(load_raw(c0 + STAGES - 1));
+        int r_next = load_raw(c0 + STAGES);
 
         for (int c = c0; c < c1; ++c) {
             issue(c + STAGES - 1, t_next);
-            t_next = load_idx(c + STAGES);
+            t_next = map_idx(r_next);
+            r_next = load_raw(c + STAGES + 1);
             cp_async_wait<STAGES - 1>();
             __syncwarp();
             const int s = (SPLIT ? c - c0 : c) % STAGES;
@@ -278,13 +285,19 @@ __global__ void __launch_bounds__(WARPS * 32)
                 plo[mt][0] = movm_t(l01);
                 plo[mt][1] = movm_t(l23);
             }
-            // ---- O^T = alpha * O^T + V^T P
+            // ---- O^T = alpha * O^T + V^T P; the rescale is skipped (exactly: alpha == 1) while no
+            // head's running max moved
+            if (__any_sync(0xffffffffu, (alpha[0] != 1.f) | (alpha[1] != 1.f))) {
+#pragma unroll
+                for (int dt = 0; dt < D / 16; ++dt) {
+                    o[dt][0] *= alpha[0];
+                    o[dt][1] *= alpha[1];
+                    o[dt][2] *= alpha[0];
+                    o[dt][3] *= alpha[1];
+                }
+            }
 #pragma unroll
             for (int dt = 0; dt < D / 16; ++dt) {
-                o[dt][0] *= alpha[0];
-                o[dt][1] *= alpha[1];
-                o[dt][2] *= alpha[0];
-                o[dt][3] *= alpha[1];
 #pragma unroll
                 for (int ks = 0; ks < MT; ++ks) {
                     uint32_t a0, a1, a2, a3;
@@ -399,23 +412,44 @@ __global__ void attn_merge_kernel(const float* __restrict__ part, int G, int spl
     }
 }
 
-// Warps per CTA of the two dense configurations (one CTA per SM fits in shared memory).
+// Warps per CTA of the dense configurations (one CTA per SM fits in shared memory).  With fewer
+// (row, KV head) units than warps on the GPU (decode), d = 128 runs 32-key chunks over 7 warps:
+// fewer, longer steps per warp, measured faster on B200 for 64 sequences x 4 KV heads.
 static constexpr int kAttnWarpsD128 = 14;
 static constexpr int kAttnWarpsD64 = 16;
+static constexpr int kAttnDecodeChunkD128 = 32;
+static constexpr int kAttnDecodeWarpsD128 = 7;
+// fp8 K/V (d = 128): 3 stages of 16-key chunks over 14 warps
+static constexpr int kAttnFp8StagesD128 = 3;
+static constexpr int kAttnFp8WarpsD128 = 14;
+static constexpr int kAttnFp8StagesD64 = 4;
+static constexpr int kAttnFp8WarpsD64 = 16;
 
-// Ranges per unit: 1 unless there are too few (row, KV head) units to give every warp of the
-// GPU two work items.  Depends only on the shape and SM count, so the workspace query and the
-// launch agree.
+static bool attn_decode_shape(long long units, int d, int num_sms) {
+    return d == 128 && units < static_cast<long long>(num_sms) * kAttnWarpsD128;
+}
+
+// Ranges per unit: 1 when the (row, KV head) units alone give every warp of the GPU (one CTA
+// per SM) work.  Otherwise each warp takes work items (unit, range) in turn, so the busiest warp
+// handles ceil(units * s / warps) items of ceil(nchunks / s) chunks; the count s (at most 32,
+// one lane per range in the merge) that makes this smallest is taken, the smallest such s on
+// ties (fewer ranges: fewer pipeline starts, a smaller merge).  Depends only on the shape and
+// SM count, so the workspace query and the launch agree.
 static int attn_splits(long long units, int nchunks, int warps, int num_sms, int* per) {
-    const long long want = 2ll * num_sms * warps;
-    int s = 1;
-    if (units < want) {
-        s = static_cast<int>((want + units - 1) / units);
-        const int most = nchunks / 4 > 1 ? nchunks / 4 : 1;  // at least 4 chunks per range
-        if (s > most) s = most;
+    const long long tw = static_cast<long long>(num_sms) * warps;
+    int best = 1;
+    long long best_cost = -1;
+    for (int s = 1; s <= 32 && s <= nchunks && (s == 1 || units < tw); ++s) {
+        const int p = (nchunks + s - 1) / s;
+        if ((nchunks + p - 1) / p != s) continue;  // this s makes the same ranges as a smaller one
+        const long long cost = ((units * s + tw - 1) / tw) * p;
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
     }
-    *per = (nchunks + s - 1) / s;
-    return (nchunks + *per - 1) / *per;
+    *per = (nchunks + best - 1) / best;
+    return best;
 }
 
 template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ = false, bool QK_SPLIT = false>
@@ -456,8 +490,7 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
                                                                    scale_log2, O, splits, per, part, share, pg, hdr);
     if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
     const int G = Hq / Hkv;
-    // splits <= 32: attn_splits keeps at least 4 of the (at most 128) 16-key chunks in a range
-    if (splits > 32) return cudaErrorInvalidValue;
+    if (splits > 32) return cudaErrorInvalidValue;  // attn_splits makes at most 32
     if (out_bf16)
         attn_merge_kernel<D, true><<<static_cast<unsigned>(units), G * 32, 0, stream>>>(part, G, splits, Hq, Hkv, O);
     else
@@ -478,8 +511,10 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
 //     ldmatrix.trans (pairs of bytes as 16-bit elements), regroups the bytes so each register
 //     holds two keys of one d, and widens them; rows of O^T (d) come out interleaved (even d,
 //     then odd d, per 16) and are written back in place.
-//   * The K scale multiplies the fp32 score; V is widened times its key's scale in fp16 (one
-//     rounding of code x fp16(scale)); P is split into fp16 hi + lo parts.
+//   * The K scale multiplies the fp32 score.  The V scale goes into the weights instead of the
+//     rows: P'[key] = p x vs[key] / vmax with vmax the largest V scale of the range so far, so
+//     P' stays in [0, 1] and its fp16 hi + lo parts keep ~22 bits; O^T is held in units of vmax
+//     (rescaled when a larger scale arrives) and the V codes widen to fp16 exactly.
 // The split rule (and so the workspace) is the bf16 kernel's for the same d.
 template <int D, int STAGES, int WARPS>
 struct Fp8AttnCfg {
@@ -516,15 +551,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
     const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
-__device__ __forceinline__ uint32_t hmul2_u32(uint32_t x, __half2 s) {
-    __half2 v = __hmul2(*reinterpret_cast<__half2*>(&x), s);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
 
 template <int D, int STAGES, int WARPS, bool OUT_BF16, bool SPLIT>
 __global__ void __launch_bounds__(WARPS * 32, 1)
@@ -553,8 +579,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     const int c4 = lane & 3;
     const int hc = 2 * c4;              // first of the two head columns this lane owns in C tiles
     const int seg = lane % C::SEG8, sub = lane / C::SEG8;
-    // ldmatrix.x4.trans over V: matrices (keys 0-7 | keys 8-15) x (segment dt | dt + 1)
+    // ldmatrix.x4 over K (and .trans over V): matrices (keys 0-7 | keys 8-15) x (segment | + 1)
     const int v_key = ((lane >> 3) & 1) * 8 + (lane & 7), v_seg = lane >> 4;
+    const int k_row = v_key, k_sg = v_seg;
 
     for (long long it = static_cast<long long>(blockIdx.x) * WARPS + warp; it < items;
          it += static_cast<long long>(gridDim.x) * WARPS) {
@@ -640,6 +667,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #pragma unroll
         for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
         float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
+        float vmax = 0.f, rvmax = 0.f;  // largest |V scale| of the range so far (O^T is held in its units)
 
         __syncwarp();
 #pragma unroll
@@ -659,18 +687,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             const int* si = srow + s * CHUNK;
             const float* ks_ = sks + s * CHUNK;
             const float* vs_ = svs + s * CHUNK;
-            // ---- S^T = K Q^T: A rows qn and qn + 8 take code bytes 16 ks + 4 c4 .. + 3
+            // ---- S^T = K Q^T: A rows qn and qn + 8 take code bytes 16 ks + 4 c4 .. + 3; one
+            // ldmatrix.x4 (8 rows x 16 bytes per matrix) delivers them for two k-steps
             float sacc[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t w0 = lds32(kst + C::at(qn, ks) + 4 * c4);
-                const uint32_t w1 = lds32(kst + C::at(qn + 8, ks) + 4 * c4);
-                const uint32_t a0 = e4m3x2_to_f16x2(w0), a2 = e4m3x2_to_f16x2(w0 >> 16);
-                const uint32_t a1 = e4m3x2_to_f16x2(w1), a3 = e4m3x2_to_f16x2(w1 >> 16);
-                if (ks & 1)
-                    mma_f16(s2, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-                else
-                    mma_f16(sacc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+            for (int ks = 0; ks < D / 16; ks += 2) {
+                uint32_t w[4];  // key rows qn / qn + 8 at k-step ks, then at ks + 1
+                ldsm_x4(kst + C::at(k_row, ks + k_sg), w[0], w[1], w[2], w[3]);
+                mma_f16(sacc, e4m3x2_to_f16x2(w[0]), e4m3x2_to_f16x2(w[1]), e4m3x2_to_f16x2(w[0] >> 16),
+                        e4m3x2_to_f16x2(w[1] >> 16), qf[ks][0], qf[ks][1]);
+                mma_f16(s2, e4m3x2_to_f16x2(w[2]), e4m3x2_to_f16x2(w[3]), e4m3x2_to_f16x2(w[2] >> 16),
+                        e4m3x2_to_f16x2(w[3] >> 16), qf[ks + 1][0], qf[ks + 1][1]);
             }
             // ---- mask, K scale, softmax scale, online softmax
             const bool v0 = si[qn] >= 0, v1 = si[qn + 8] >= 0;
@@ -684,16 +711,33 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
             }
+            // V scales fold into the weights: P'[key] = p * vs[key] / vmax, in [0, 1], so its fp16
+            // hi + lo parts keep ~22 bits; when a chunk brings a larger scale, O^T (held in units
+            // of vmax) is rescaled like the running max's alpha.
+            const float vq0 = vs_[qn], vq1 = vs_[qn + 8];
+            float cmax = fmaxf(fabsf(vq0), fabsf(vq1));
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, off));
+            float beta = 1.f;
+            if (cmax > vmax) {  // warp-uniform: every lane holds the same cmax and vmax
+                beta = vmax / cmax;
+                vmax = cmax;
+                rvmax = 1.f / cmax;
+            }
+            const float u0 = vq0 * rvmax, u1 = vq1 * rvmax;
             float alpha[2], mnew[2], p[4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 mnew[j] = fmaxf(mrun[j], mx[j]);
-                alpha[j] = (mnew[j] == -INFINITY) ? 1.f : exp2f(mrun[j] - mnew[j]);
+                const float a = (mnew[j] == -INFINITY) ? 1.f : exp2f(mrun[j] - mnew[j]);
                 mrun[j] = mnew[j];
-                lrun[j] *= alpha[j];
-                p[j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[j] - mnew[j]);
-                p[2 + j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[2 + j] - mnew[j]);
-                lrun[j] += p[j] + p[2 + j];
+                lrun[j] *= a;
+                alpha[j] = a * beta;
+                const float e0 = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[j] - mnew[j]);
+                const float e1 = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[2 + j] - mnew[j]);
+                lrun[j] += e0 + e1;
+                p[j] = e0 * u0;
+                p[2 + j] = e1 * u1;
             }
             const uint32_t h01 = pack_f16(p[0], p[1]);
             const uint32_t h23 = pack_f16(p[2], p[3]);
@@ -702,10 +746,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             const uint32_t phi0 = movm_t(h01), phi1 = movm_t(h23);
             const uint32_t plo0 = movm_t(pack_f16(p[0] - r01.x, p[1] - r01.y));
             const uint32_t plo1 = movm_t(pack_f16(p[2] - r23.x, p[3] - r23.y));
-            // V scales of the keys this lane's A elements hold: 2 c4, 2 c4 + 1 and 8 + 2 c4, 9 + 2 c4
-            const __half2 vs_lo = __floats2half2_rn(vs_[2 * c4], vs_[2 * c4 + 1]);
-            const __half2 vs_hi = __floats2half2_rn(vs_[8 + 2 * c4], vs_[9 + 2 * c4]);
-            // ---- O^T = alpha * O^T + V^T P, two 16-d blocks per ldmatrix.x4.trans
+            // ---- O^T = alpha * O^T + V^T P, two 16-d blocks per ldmatrix.x4.trans (rescale skipped
+            // while no head's running max moved: alpha == 1 exactly)
+            if (__any_sync(0xffffffffu, (alpha[0] != 1.f) | (alpha[1] != 1.f))) {
+#pragma unroll
+                for (int dt = 0; dt < D / 16; ++dt) {
+                    o[dt][0] *= alpha[0];
+                    o[dt][1] *= alpha[1];
+                    o[dt][2] *= alpha[0];
+                    o[dt][3] *= alpha[1];
+                }
+            }
 #pragma unroll
             for (int dt = 0; dt < D / 16; dt += 2) {
                 uint32_t r[4];
@@ -715,15 +766,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     // r[2e]: keys 0-7, r[2e+1]: keys 8-15; bytes (k0,d) (k0,d+1) (k1,d) (k1,d+1)
                     const uint32_t lo = __byte_perm(r[2 * e], 0u, 0x3120);
                     const uint32_t hi = __byte_perm(r[2 * e + 1], 0u, 0x3120);
-                    const uint32_t a0 = hmul2_u32(e4m3x2_to_f16x2(lo), vs_lo);        // d even
-                    const uint32_t a1 = hmul2_u32(e4m3x2_to_f16x2(lo >> 16), vs_lo);  // d odd
-                    const uint32_t a2 = hmul2_u32(e4m3x2_to_f16x2(hi), vs_hi);
-                    const uint32_t a3 = hmul2_u32(e4m3x2_to_f16x2(hi >> 16), vs_hi);
+                    const uint32_t a0 = e4m3x2_to_f16x2(lo);        // d even
+                    const uint32_t a1 = e4m3x2_to_f16x2(lo >> 16);  // d odd
+                    const uint32_t a2 = e4m3x2_to_f16x2(hi);
+                    const uint32_t a3 = e4m3x2_to_f16x2(hi >> 16);
                     float(&od)[4] = o[dt + e];
-                    od[0] *= alpha[0];
-                    od[1] *= alpha[1];
-                    od[2] *= alpha[0];
-                    od[3] *= alpha[1];
                     mma_f16(od, a0, a1, a2, a3, phi0, phi1);
                     mma_f16(od, a0, a1, a2, a3, plo0, plo1);
                 }
@@ -745,7 +792,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int h = hc + j;
-                    if (h < G) *reinterpret_cast<float2*>(pb + h * (D + 2) + d0) = make_float2(o[dt][j], o[dt][2 + j]);
+                    if (h < G)
+                        *reinterpret_cast<float2*>(pb + h * (D + 2) + d0) =
+                            make_float2(o[dt][j] * vmax, o[dt][2 + j] * vmax);
                 }
             }
             if (qn == 0) {
@@ -760,8 +809,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             }
             continue;
         }
-        const float inv0 = lrun[0] > 0.f ? 1.f / lrun[0] : 0.f;
-        const float inv1 = lrun[1] > 0.f ? 1.f / lrun[1] : 0.f;
+        const float inv0 = lrun[0] > 0.f ? vmax / lrun[0] : 0.f;
+        const float inv1 = lrun[1] > 0.f ? vmax / lrun[1] : 0.f;
 #pragma unroll
         for (int dt = 0; dt < D / 16; ++dt) {
             const int d0 = dt * 16 + 2 * qn;
@@ -785,7 +834,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
     }
 }
 
-template <int D, int STAGES, int WARPS, int SPLIT_WARPS>
+template <int D, int STAGES, int WARPS>
 static cudaError_t launch_attn_fp8_t(const __nv_bfloat16* Q, const unsigned char* K8, const float* k_scale,
                                      const unsigned char* V8, const float* v_scale, const int* idx, int B, int Hq,
                                      int Hkv, int topk, float scale, void* O, bool out_bf16, KvPages pg, WsHeader* hdr,
@@ -794,8 +843,7 @@ static cudaError_t launch_attn_fp8_t(const __nv_bfloat16* Q, const unsigned char
     const long long units = static_cast<long long>(B) * Hkv;
     const int nchunks = (topk + C::CHUNK - 1) / C::CHUNK;
     int per = nchunks;
-    // the bf16 kernel's split rule for this d, so sparse_attn_part_bytes sizes the workspace
-    const int splits = attn_splits(units, nchunks, SPLIT_WARPS, num_sms, &per);
+    const int splits = attn_splits(units, nchunks, WARPS, num_sms, &per);
     using KernFn = void (*)(const __nv_bfloat16*, const unsigned char*, const float*, const unsigned char*,
                             const float*, const int*, int, int, int, int, float, void*, int, int, float*, KvPages,
                             WsHeader*);
@@ -823,13 +871,21 @@ static cudaError_t launch_attn_fp8_t(const __nv_bfloat16* Q, const unsigned char
     return cudaGetLastError();
 }
 
-// Bytes of split-range state the sparse attention needs beyond the status word.
+// Bytes of split-range state the sparse attention needs beyond the status word: the larger of
+// the bf16 kernel's and (one query per sequence) the fp8 kernel's ranges for this shape.
 size_t sparse_attn_part_bytes(int B, int n_q, int Hq, int Hkv, int d, int topk, int num_sms) {
     if (d != 128 && d != 64) return 0;
-    const int warps = d == 128 ? kAttnWarpsD128 : kAttnWarpsD64;
     const long long units = static_cast<long long>(B) * n_q * Hkv;
     int per = 0;
-    const int splits = attn_splits(units, (topk + 15) / 16, warps, num_sms, &per);
+    const bool dec = attn_decode_shape(units, d, num_sms);
+    const int chunk = dec ? kAttnDecodeChunkD128 : 16;
+    const int warps = dec ? kAttnDecodeWarpsD128 : d == 128 ? kAttnWarpsD128 : kAttnWarpsD64;
+    int splits = attn_splits(units, (topk + chunk - 1) / chunk, warps, num_sms, &per);
+    if (n_q == 1) {
+        const int s8 = attn_splits(units, (topk + 15) / 16, d == 128 ? kAttnFp8WarpsD128 : kAttnFp8WarpsD64, num_sms,
+                                   &per);
+        if (s8 > splits) splits = s8;
+    }
     if (splits == 1) return 0;
     return static_cast<size_t>(units) * splits * (Hq / Hkv) * (d + 2) * sizeof(float);
 }
@@ -842,7 +898,12 @@ cudaError_t launch_sparse_attn(const void* Q, const void* K, const void* V, cons
     auto k = static_cast<const __nv_bfloat16*>(K);
     auto v = static_cast<const __nv_bfloat16*>(V);
     // 16-key chunks, 2 stages per warp, swizzled rows: as many warps per SM as shared memory
-    // holds (measured on B200: warps in flight matter more than stages per warp).
+    // holds (measured on B200: warps in flight matter more than stages per warp); 32-key
+    // chunks for decode shapes at d = 128.
+    const long long units = static_cast<long long>(B) * n_q * Hkv;
+    if (d == 128 && attn_decode_shape(units, d, num_sms))
+        return launch_attn_t<128, kAttnDecodeChunkD128, 2, kAttnDecodeWarpsD128, true, true>(
+            q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O, out_bf16, share, pg, hdr, num_sms, stream);
     if (d == 128)
         return launch_attn_t<128, 16, 2, kAttnWarpsD128, true, true>(q, k, v, idx, B, n_q, n_kv, Hq, Hkv, topk, scale, O,
                                                          out_bf16, share, pg, hdr, num_sms, stream);
@@ -860,13 +921,13 @@ cudaError_t launch_sparse_attn_fp8_paged(const void* Q, const void* K8, const fl
     auto q = static_cast<const __nv_bfloat16*>(Q);
     auto k = static_cast<const unsigned char*>(K8);
     auto v = static_cast<const unsigned char*>(V8);
-    // 3 stages of 4 KB codes per warp: 16 warps per SM at d = 128
     if (d == 128)
-        return launch_attn_fp8_t<128, 3, 16, kAttnWarpsD128>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale,
-                                                              O, out_bf16, pg, hdr, num_sms, stream);
+        return launch_attn_fp8_t<128, kAttnFp8StagesD128, kAttnFp8WarpsD128>(
+            q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale, O, out_bf16, pg, hdr, num_sms, stream);
     if (d == 64)
-        return launch_attn_fp8_t<64, 4, 16, kAttnWarpsD64>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv, topk, scale, O,
-                                                            out_bf16, pg, hdr, num_sms, stream);
+        return launch_attn_fp8_t<64, kAttnFp8StagesD64, kAttnFp8WarpsD64>(q, k, k_scale, v, v_scale, idx, B, Hq, Hkv,
+                                                                         topk, scale, O, out_bf16, pg, hdr, num_sms,
+                                                                         stream);
     return cudaErrorNotSupported;
 }
 

@@ -169,7 +169,7 @@ def test_latent_attention_matches_oracle(case):
 SHARED = [
     ("mtp4_gqa", 3, 4, 2996, 3000, 32, 4, 128, 2048, 4),
     ("mtp_ragged_d64", 2, 5, 995, 1000, 16, 2, 64, 300, 2),
-    ("mtp_b64_split_ranges", 64, 4, 1996, 2000, 32, 4, 128, 512, 4),
+    ("mtp_b64", 64, 4, 1996, 2000, 32, 4, 128, 512, 4),
     ("mtp_latent", 2, 3, 497, 500, 16, 1, 576, 128, 3),
 ]
 
