@@ -657,10 +657,27 @@ def run_profile_paged(args):
         if it >= args.warmup:
             t_b.append(e[0].elapsed_time(e[1]))
             t_8.append(e[1].elapsed_time(e[2]))
+    # steady state: 10 back-to-back calls per event pair behind an untimed one, so the host's
+    # launch work overlaps the GPU (a single call after a synchronize times the host too)
+    def burst(fn, n=10):
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+    tb = min(burst(lambda: dsa.sparse_attn_topk_paged(Q, Kp, Vp, table, seq, idx, o_dtype=torch.bfloat16, out=O,
+                                                      workspace=ws)) for _ in range(3))
+    t8 = min(burst(lambda: dsa.sparse_attn_topk_paged_e4m3(Q, K8, ks, V8, vs, table, seq, idx,
+                                                           o_dtype=torch.bfloat16, out=O, workspace=ws))
+             for _ in range(3))
     dsa.check_status(ws)
     by = B * TOPK * HKV * DH * 2          # K and V codes gathered (bf16: twice this)
-    print(json.dumps({"case": "profile_paged", "bf16_ms": min(t_b), "bf16_gathered_gbs": 2 * by / min(t_b) / 1e6,
-                      "fp8_ms": min(t_8), "fp8_gathered_gbs": by / min(t_8) / 1e6}))
+    print(json.dumps({"case": "profile_paged", "bf16_ms": tb, "bf16_gathered_gbs": 2 * by / tb / 1e6,
+                      "fp8_ms": t8, "fp8_gathered_gbs": by / t8 / 1e6, "fp8_over_bf16": t8 / tb,
+                      "single_call_bf16_ms": min(t_b), "single_call_fp8_ms": min(t_8)}))
 
 
 def run_profile_latent(args):

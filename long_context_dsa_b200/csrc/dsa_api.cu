@@ -378,7 +378,7 @@ int sparse_attn_topk_paged(const void* Q, const void* K_pages, const void* V_pag
                     num_pages, max_pages);
     const long long pool = static_cast<long long>(num_pages) * page_size;
     if (pool > 0x7fffffffll) return fail(DSA_ERR_INVALID_ARG, "page pool too large");
-    const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages};
+    const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages, dsa::page_shift_of(page_size)};
     return attn_common(Q, K_pages, V_pages, idx, B, 1, static_cast<int>(pool), Hq, Hkv, d, d, topk, scale, O,
                        o_dtype, dsa::kNoShare, workspace, workspace_bytes, stream, pages);
 }
@@ -408,7 +408,7 @@ int sparse_attn_topk_paged_e4m3(const void* Q, const void* K8_pages, const float
     if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(d));
     int sms;
     if ((rc = sm_count(&sms))) return rc;
-    const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages};
+    const dsa::KvPages pages = {page_table, seq_lens, page_size, max_pages, num_pages, dsa::page_shift_of(page_size)};
     cudaError_t e = launch_sparse_attn_fp8_paged(Q, K8_pages, k_scale, V8_pages, v_scale, idx, B, Hq, Hkv, d, topk,
                                                  scale, O, o_dtype == DSA_BF16, pages,
                                                  static_cast<WsHeader*>(workspace), sms,

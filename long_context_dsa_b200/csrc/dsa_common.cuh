@@ -57,8 +57,20 @@ struct KvPages {
     const int* table;
     const int* lens;
     int page_size, max_pages, num_pages;
+    int page_shift;  // log2(page_size) when it is a power of two, else -1 (shift / mask instead of divide)
+    __device__ __forceinline__ int page_of(int t) const { return page_shift >= 0 ? t >> page_shift : t / page_size; }
+    __device__ __forceinline__ int in_page(int t) const {
+        return page_shift >= 0 ? t & (page_size - 1) : t % page_size;
+    }
 };
-static constexpr KvPages kContiguous = {nullptr, nullptr, 0, 0, 0};
+static constexpr KvPages kContiguous = {nullptr, nullptr, 0, 0, 0, -1};
+// log2 of a power-of-two page size, -1 for any other size
+inline int page_shift_of(int page_size) {
+    if (page_size < 1 || (page_size & (page_size - 1)) != 0) return -1;
+    int s = 0;
+    while ((1 << s) < page_size) ++s;
+    return s;
+}
 
 // Nanoseconds from the global timer.
 __device__ __forceinline__ uint64_t globaltimer_ns() {

@@ -152,12 +152,12 @@ __global__ void __launch_bounds__(WARPS * 32)
             }
             if (SHARED && t > lim) t = -1;
             if (PAGED && t >= 0) {
-                const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + t / pg.page_size);
+                const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + pg.page_of(t));
                 if (page < 0 || page >= pg.num_pages) {
                     raise_status(hdr, DSA_STATUS_BAD_INDEX, page);
                     t = -1;
                 } else {
-                    t = page * pg.page_size + t % pg.page_size;
+                    t = page * pg.page_size + pg.in_page(t);
                 }
             }
             return t;
@@ -546,10 +546,12 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
-// two E4M3 codes (low byte first) -> two fp16 values, exactly
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// four E4M3 codes (low byte first) -> bytes 0-1 and bytes 2-3 as two pairs of fp16 values, exactly
+// (the word is split into its 16-bit halves in registers, no shift)
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(four));
 }
 
 template <int D, int STAGES, int WARPS, bool OUT_BF16, bool SPLIT>
@@ -609,12 +611,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                 t = -1;
             }
             if (t >= 0) {
-                const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + t / pg.page_size);
+                const int page = __ldg(pg.table + static_cast<size_t>(b) * pg.max_pages + pg.page_of(t));
                 if (page < 0 || page >= pg.num_pages) {
                     raise_status(hdr, DSA_STATUS_BAD_INDEX, page);
                     t = -1;
                 } else {
-                    t = page * pg.page_size + t % pg.page_size;
+                    t = page * pg.page_size + pg.in_page(t);
                 }
             }
             return t;
@@ -694,10 +696,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
             for (int ks = 0; ks < D / 16; ks += 2) {
                 uint32_t w[4];  // key rows qn / qn + 8 at k-step ks, then at ks + 1
                 ldsm_x4(kst + C::at(k_row, ks + k_sg), w[0], w[1], w[2], w[3]);
-                mma_f16(sacc, e4m3x2_to_f16x2(w[0]), e4m3x2_to_f16x2(w[1]), e4m3x2_to_f16x2(w[0] >> 16),
-                        e4m3x2_to_f16x2(w[1] >> 16), qf[ks][0], qf[ks][1]);
-                mma_f16(s2, e4m3x2_to_f16x2(w[2]), e4m3x2_to_f16x2(w[3]), e4m3x2_to_f16x2(w[2] >> 16),
-                        e4m3x2_to_f16x2(w[3] >> 16), qf[ks + 1][0], qf[ks + 1][1]);
+                uint32_t a[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) e4m3x4_to_f16x2x2(w[i], a[2 * i], a[2 * i + 1]);
+                // A fragment (a0, a1, a2, a3) = (row qn bytes 0-1, row qn + 8 bytes 0-1, row qn bytes 2-3, ...)
+                mma_f16(sacc, a[0], a[2], a[1], a[3], qf[ks][0], qf[ks][1]);
+                mma_f16(s2, a[4], a[6], a[5], a[7], qf[ks + 1][0], qf[ks + 1][1]);
             }
             // ---- mask, K scale, softmax scale, online softmax
             const bool v0 = si[qn] >= 0, v1 = si[qn + 8] >= 0;
@@ -766,10 +770,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
                     // r[2e]: keys 0-7, r[2e+1]: keys 8-15; bytes (k0,d) (k0,d+1) (k1,d) (k1,d+1)
                     const uint32_t lo = __byte_perm(r[2 * e], 0u, 0x3120);
                     const uint32_t hi = __byte_perm(r[2 * e + 1], 0u, 0x3120);
-                    const uint32_t a0 = e4m3x2_to_f16x2(lo);        // d even
-                    const uint32_t a1 = e4m3x2_to_f16x2(lo >> 16);  // d odd
-                    const uint32_t a2 = e4m3x2_to_f16x2(hi);
-                    const uint32_t a3 = e4m3x2_to_f16x2(hi >> 16);
+                    uint32_t a0, a1, a2, a3;  // a0 / a2: d even, a1 / a3: d odd
+                    e4m3x4_to_f16x2x2(lo, a0, a1);
+                    e4m3x4_to_f16x2x2(hi, a2, a3);
                     float(&od)[4] = o[dt + e];
                     mma_f16(od, a0, a1, a2, a3, phi0, phi1);
                     mma_f16(od, a0, a1, a2, a3, plo0, plo1);
