@@ -165,9 +165,9 @@ def pattern_search(layers, dev, rows=2048, n_f=2):
 
 def attn_traffic():
     """DRAM bytes of one full sparse-attention launch, scaled from the ncu capture of the tail case
-    (4096 rows x 2048 selected keys: 2.492 GB read + 0.037 GB written) by selected (query, key) pairs;
+    (4096 rows x 2048 selected keys: 2.981 GB read + 0.036 GB written) by selected (query, key) pairs;
     an over-estimate (earlier rows hit L2 more).  Update with the capture when the kernel changes."""
-    per_pair = (2.491670e9 + 0.036963e9) / (4096 * 2048)
+    per_pair = (2.981177e9 + 0.035541e9) / (4096 * 2048)
     pairs = sum(min(TOPK, t + 1) for t in range(L))
     return round(per_pair * pairs)
 
