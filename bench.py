@@ -740,6 +740,36 @@ def run_profile_decode1m(args):
     print(json.dumps({"case": "profile_decode1m", "ms": min(ts), "key_gbs": n * (D_I + 4) / min(ts) / 1e6}))
 
 
+def run_profile_decode(args):
+    """One decode indexer call of the batched decode shape for ncu captures: 64 sequences, one
+    query each at the end of a 200000-token bf16 key cache (H_I=32, d_I=128, top-2048): the split
+    decode kernel writing every row's score keys, then the radix select."""
+    import torch
+    from long_context_dsa_b200 import dsa, synth
+
+    dev = torch.device("cuda", 0)
+    B, Lc = 64, 200000
+    gen = synth.StructuredIndexer("decode200k", B, Lc, H_I, D_I, r=32, base_std=1.0, noise_std=SIGMA_200K,
+                                  device=dev, seed=2000)
+    q, w = gen.queries(0, Lc - 1, Lc)
+    k = gen.keys(0)
+    del gen
+    ws = torch.zeros(dsa.idx_score_topk_workspace_size(B, 1, Lc - 1, Lc, H_I, D_I, TOPK), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((B, 1, TOPK), dtype=torch.int32, device=dev)
+    ts = []
+    for it in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dsa.idx_score_topk(q, k, w, TOPK, q_pos0=Lc - 1, out=out, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    dsa.check_status(ws)
+    print(json.dumps({"case": "profile_decode", "ms": min(ts), "key_gbs": B * Lc * D_I * 2 / min(ts) / 1e6}))
+
+
 def run_decode(args, dev):
     """Decode step: 64 sequences, one new token each, at a 200000-token cache; 4 layers FSSS
     (H_I=32, d_I=128, top-2048; attention 32 query / 4 KV heads, d=128)."""
@@ -1480,7 +1510,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the decode and 1M-chunk measurements")
     ap.add_argument("--case", default="bench",
                     choices=["bench", "profile", "profile_paged", "decode", "decode_mha", "ctx1m", "mtp", "paged",
-                             "prefill16k", "decode1m", "ctx1m_full", "profile_latent", "profile_decode1m", "cp"],
+                             "prefill16k", "decode1m", "ctx1m_full", "profile_latent", "profile_decode1m", "profile_decode",
+                             "cp"],
                     help="profile: small single-kernel launches for ncu captures; decode / ctx1m / ...: only "
                          "that extra measurement, printed as one JSON line; cp: one 200K sequence split over "
                          "the torchrun ranks (context-parallel prefill, strong scaling)")
@@ -1490,6 +1521,9 @@ def main():
         return
     if args.case == "profile_paged":
         run_profile_paged(args)
+        return
+    if args.case == "profile_decode":
+        run_profile_decode(args)
         return
     if args.case == "profile_latent":
         run_profile_latent(args)

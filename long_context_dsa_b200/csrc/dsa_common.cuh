@@ -19,7 +19,9 @@ struct WsHeader {
     int status;        // DSA_STATUS_* bits, OR-ed by kernels
     int detail;        // first offending value (bad index) or wait site
     int test_hook;     // DSA_TEST_WITHHOLD_TILE: the TMA producers withhold their first key tile
-    int pad[61];
+    int sel_full_rows;  // decode rows whose bin select fell back to the whole row (statistics)
+    int sel_max_kept;   // most keys a decode row's bin select kept (statistics)
+    int pad[59];
 };
 static constexpr size_t kWsHeaderBytes = 256;
 
@@ -71,6 +73,10 @@ inline int page_shift_of(int page_size) {
     while ((1 << s) < page_size) ++s;
     return s;
 }
+
+// Top bits of an order-preserving score key that the one-query decode indexer counts into a
+// per-row histogram for the bin select that follows it (sign, 8 exponent bits, 4 mantissa bits).
+static constexpr int kBinTopkBits = 13;
 
 // Nanoseconds from the global timer.
 __device__ __forceinline__ uint64_t globaltimer_ns() {

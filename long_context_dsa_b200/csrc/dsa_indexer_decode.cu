@@ -29,6 +29,10 @@ namespace dsa {
 
 cudaError_t launch_topk_merge_pairs(const uint32_t* keys, const int* idxs, int rows, int len, int k, int* out,
                                     WsHeader* hdr, int num_sms, cudaStream_t stream, int n_tok);
+size_t bin_topk_hist_bytes(int rows);
+size_t bin_topk_scratch_bytes(int rows, int n, int num_sms);
+cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
+                            WsHeader* hdr, int num_sms, cudaStream_t stream);
 size_t radix_topk_scratch_bytes(int rows, int n, int num_sms);
 cudaError_t launch_radix_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
                               int num_sms, cudaStream_t stream);
@@ -72,6 +76,7 @@ struct DecParams {
     uint32_t* part_key;  // [B * splits, topk]
     int* part_idx;       // [B * splits, topk]
     uint32_t* score_keys;  // [B, q_pos0 + 1] order-preserving score keys (score mode), or NULL
+    int* hist;             // score mode: [B, 2^kBinTopkBits] counts of the keys' top bits (zeroed before)
     WsHeader* hdr;
 };
 
@@ -263,6 +268,10 @@ __global__ void __launch_bounds__(192, 1)
                 ws[tid] = wv;
             }
             if (tid == 0) topk_row_init(st);
+            // score mode: the unit's histogram of its keys' top bits lives where the candidates would
+            int* shist = reinterpret_cast<int*>(ckey);  // 2^kBinTopkBits counts in the ckey + cidx region
+            if (p.score_keys)
+                for (int i = tid; i < (1 << kBinTopkBits); i += 128) shist[i] = 0;
             grp.sync();
             int cnt = 0;
             uint32_t* wkey = ckey + warp * sub;
@@ -302,8 +311,11 @@ __global__ void __launch_bounds__(192, 1)
                 if (FP8) sc_v *= ksc;
                 const uint32_t key = score_key(sc_v);
                 if (p.score_keys) {
-                    // score mode: the row's keys go to memory and a multi-CTA radix select picks the top-k
-                    if (got && s_key < len) p.score_keys[static_cast<size_t>(b) * (p.q_pos0 + 1) + s_key] = key;
+                    // score mode: the row's keys go to memory and into the histogram of their top bits;
+                    // the bin select picks the top-k
+                    const bool v = got && s_key < len;
+                    if (v) p.score_keys[static_cast<size_t>(b) * (p.q_pos0 + 1) + s_key] = key;
+                    if (v) atomicAdd(&shist[key >> (32 - kBinTopkBits)], 1);
                 } else {
                     const uint32_t tk = st->thr_key;
                     const bool adm = got & (s_key < len) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
@@ -328,7 +340,45 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             if (!ok) break;
-            if (p.score_keys) continue;
+            if (p.score_keys) {
+                grp.sync();  // every key of the unit is counted
+                // Only the bins from this unit's own k-th key up go to the row's histogram: the unit
+                // alone holds k keys at or above that bin, so the row's k-th key lies there too, and
+                // every bin the row's threshold search looks at still gets all its counts.
+                constexpr int NB = 1 << kBinTopkBits, PB = NB / 128;
+                int cs = 0;
+                for (int j = 0; j < PB; ++j) cs += shist[tid * PB + j];
+                int suf = cs;  // keys in bins >= tid * PB, first within the warp
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int o = __shfl_down_sync(0xffffffffu, suf, off);
+                    if (lane + off < 32) suf += o;
+                }
+                if (lane == 0) sortbuf[warp] = suf;
+                if (tid == 0) sortbuf[4] = 0;
+                grp.sync();
+                for (int ww = warp + 1; ww < 4; ++ww) suf += sortbuf[ww];
+                if (suf >= p.topk && suf - cs < p.topk) {
+                    int acc = suf - cs, T = tid * PB;
+                    for (int j = PB - 1; j >= 0; --j) {
+                        acc += shist[tid * PB + j];
+                        if (acc >= p.topk) {
+                            T = tid * PB + j;
+                            break;
+                        }
+                    }
+                    sortbuf[4] = T;
+                }
+                grp.sync();
+                const int t_lo = sortbuf[4];
+                int* gh = p.hist + static_cast<size_t>(b) * NB;
+                for (int i = t_lo + tid; i < NB; i += 128) {
+                    const int c = shist[i];
+                    if (c) atomicAdd(gh + i, c);
+                }
+                grp.sync();  // before the next unit clears it
+                continue;
+            }
             if (lane == 0) st->cnt[warp] = cnt;
             grp.sync();
             grp.finish(st, ckey, cidx, p.topk, p.part_idx + static_cast<size_t>(u) * p.topk,
@@ -436,22 +486,24 @@ cudaError_t launch_dec_t(const void* q, const float* q_scale, const void* k, con
     p.part_key = reinterpret_cast<uint32_t*>(scratch);
     p.part_idx = reinterpret_cast<int*>(p.part_key + parts);
     p.score_keys = nullptr;
+    p.hist = nullptr;
+    const size_t keys_bytes = (static_cast<size_t>(B) * max_len * 4 + 255) / 256 * 256;
     if (radix) {
         p.part_key = nullptr;
         p.part_idx = nullptr;
         p.score_keys = reinterpret_cast<uint32_t*>(scratch);
+        p.hist = reinterpret_cast<int*>(scratch + keys_bytes);
     }
     auto kern = indexer_decode_kernel<H, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
+    if (radix && (e = cudaMemsetAsync(p.hist, 0, bin_topk_hist_bytes(B), stream)) != cudaSuccess) return e;
     const int units = B * p.splits;
     kern<<<units < num_sms ? units : num_sms, C::THREADS, C::SMEM, stream>>>(mq, mk, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (radix) {
-        const size_t keys_bytes = (static_cast<size_t>(B) * max_len * 4 + 255) / 256 * 256;
-        return launch_radix_topk(p.score_keys, max_len, B, max_len, topk, idx_out, scratch + keys_bytes, num_sms,
-                                 stream);
-    }
+    if (radix)
+        return launch_bin_topk(p.score_keys, max_len, B, max_len, topk, idx_out, scratch + keys_bytes, p.hdr,
+                               num_sms, stream);
     return launch_topk_merge_pairs(p.part_key, p.part_idx, B, p.splits * topk, topk, idx_out, p.hdr, num_sms,
                                    stream, max_len);
 }
@@ -467,9 +519,9 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
 }
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen) {
-    if (!varlen) {  // contiguous caches: the row's score keys, then the radix select's state
+    if (!varlen) {  // contiguous caches: the row's score keys, then the bin select's state
         const size_t keys_bytes = (static_cast<size_t>(B) * (q_pos0 + 1) * 4 + 255) / 256 * 256;
-        return keys_bytes + radix_topk_scratch_bytes(B, q_pos0 + 1, num_sms);
+        return keys_bytes + bin_topk_scratch_bytes(B, q_pos0 + 1, num_sms);
     }
     const int nkt = (q_pos0 + 1 + 127) / 128;  // varlen: q_pos0 = the longest sequence - 1
     int splits = dec_splits(B, nkt, num_sms, per_sm_for(B, varlen));

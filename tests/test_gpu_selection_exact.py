@@ -7,8 +7,8 @@ index, ascending output, -1 padding) leaves exactly one correct answer.  Small v
 ranges make equal scores and zero scores common, so tie-breaking, the streaming prune of
 the fused kernel (and its exact fallback when one score value holds more ties than the
 prune's slack), the split decode kernel's partial lists and both of its merges are all
-checked for exactness, not within a tolerance; so is the multi-CTA radix select that one-query
-decode over a contiguous cache uses.
+checked for exactness, not within a tolerance; so is the bin select (histogram of the score
+keys' top bits, kept keys, exact select) that one-query decode over a contiguous cache uses.
 
 [QbitAI] §IndexCache / [Term] "dot product + top-k": the selection is the k best scores
 of each query row; ties to the lower index is this library's stated rule.
@@ -143,8 +143,38 @@ def test_decode_fp8_selection_is_exact():
 
 def test_decode_long_cache_selection_is_exact():
     """One query against a 1.7M-token cache: the score keys of the whole row go through the
-    multi-CTA radix select."""
+    bin select (or, with these heavily tied scores, its whole-row fallback)."""
     _decode_case("dec_long", 1, 1_700_000, 32, 2048, -2, 2)
+
+
+def _bin_select_stats(ws):
+    """(rows selected from the whole row, most keys a row kept) recorded by the decode bin select."""
+    v = ws[12:20].cpu().view(torch.int32).tolist()
+    return v[0], v[1]
+
+
+def _decode_with_stats(name, B, n_kv, H, topk, lo, hi):
+    d = 128
+    q, k, w = synth.integer_indexer(name, B, n_kv, H, d, lo, hi, q_rows=1)
+    ws = torch.zeros(dsa.idx_score_topk_workspace_size(B, 1, n_kv - 1, n_kv, H, d, topk, dsa.DSA_BF16),
+                     dtype=torch.uint8, device=DEV)
+    idx = dsa.idx_score_topk(q.to(DEV), k.to(DEV), w.to(DEV), topk, q_pos0=n_kv - 1, workspace=ws)
+    assert dsa.read_status(ws) == 0
+    idx = idx.cpu().numpy()
+    for b in range(B):
+        sc = oracle.indexer_scores(q[b], k[b], w[b], n_kv - 1)
+        _expect_identical(idx[b], oracle.topk_select(sc, topk, n_kv - 1), f"{name} b={b}")
+    return _bin_select_stats(ws)
+
+
+def test_decode_bin_select_fast_path_and_whole_row_fallback_are_exact():
+    """The decode select keeps the keys of the k-th key's histogram bin and above and selects
+    among them; spread scores take that path, while equal scores (every key in one bin) overflow
+    the kept-key buffers and are selected from the whole row.  Both must match the oracle."""
+    full, kept = _decode_with_stats("bin_fast", 3, 30000, 32, 512, -8, 8)
+    assert full == 0 and 512 <= kept <= 16384, (full, kept)
+    full, kept = _decode_with_stats("bin_equal", 2, 30000, 32, 512, 0, 0)
+    assert full == 2, (full, kept)
 
 
 def test_paged_decode_streaming_merge_selection_is_exact():
