@@ -33,9 +33,6 @@ size_t bin_topk_hist_bytes(int rows);
 size_t bin_topk_scratch_bytes(int rows, int n, int num_sms);
 cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
                             WsHeader* hdr, int num_sms, cudaStream_t stream);
-size_t radix_topk_scratch_bytes(int rows, int n, int num_sms);
-cudaError_t launch_radix_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
-                              int num_sms, cudaStream_t stream);
 
 template <int H, bool FP8>
 struct DecCfg {
@@ -481,14 +478,14 @@ cudaError_t launch_dec_t(const void* q, const float* q_scale, const void* k, con
     p.splits = (nkt + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty units
     p.hdr = static_cast<WsHeader*>(ws);
     unsigned char* scratch = static_cast<unsigned char*>(ws) + kWsHeaderBytes;
-    const bool radix = !paged;  // contiguous caches: score keys to memory, then the radix select
+    const bool bins = !paged;  // contiguous caches: score keys and their histogram, then the bin select
     const size_t parts = static_cast<size_t>(B) * p.splits * topk;
     p.part_key = reinterpret_cast<uint32_t*>(scratch);
     p.part_idx = reinterpret_cast<int*>(p.part_key + parts);
     p.score_keys = nullptr;
     p.hist = nullptr;
     const size_t keys_bytes = (static_cast<size_t>(B) * max_len * 4 + 255) / 256 * 256;
-    if (radix) {
+    if (bins) {
         p.part_key = nullptr;
         p.part_idx = nullptr;
         p.score_keys = reinterpret_cast<uint32_t*>(scratch);
@@ -497,11 +494,11 @@ cudaError_t launch_dec_t(const void* q, const float* q_scale, const void* k, con
     auto kern = indexer_decode_kernel<H, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    if (radix && (e = cudaMemsetAsync(p.hist, 0, bin_topk_hist_bytes(B), stream)) != cudaSuccess) return e;
+    if (bins && (e = cudaMemsetAsync(p.hist, 0, bin_topk_hist_bytes(B), stream)) != cudaSuccess) return e;
     const int units = B * p.splits;
     kern<<<units < num_sms ? units : num_sms, C::THREADS, C::SMEM, stream>>>(mq, mk, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (radix)
+    if (bins)
         return launch_bin_topk(p.score_keys, max_len, B, max_len, topk, idx_out, scratch + keys_bytes, p.hdr,
                                num_sms, stream);
     return launch_topk_merge_pairs(p.part_key, p.part_idx, B, p.splits * topk, topk, idx_out, p.hdr, num_sms,

@@ -125,7 +125,7 @@ def test_indexer_survivors_concentrated_in_one_lane_range():
 
 
 def test_decode_long_cache():
-    """One query against a 1.7M-token cache (the score keys of the row, then the multi-CTA radix
+    """One query against a 1.7M-token cache (the score keys of the row, then the histogram-bin
     select); the selection follows the oracle's rule."""
     B, L, H, d, k = 1, 1_700_000, 32, 128, 2048
     g = synth.StructuredIndexer("long_decode", B, L, H, d, r=32, base_std=1.0, noise_std=0.2, seed=0)
