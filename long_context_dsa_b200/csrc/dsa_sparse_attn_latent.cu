@@ -271,21 +271,29 @@ __global__ void __launch_bounds__(WARPS * 32, 1)
 
 // Combine the split ranges of each (query row, head block): for every head,
 // O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s (a range that met only
-// skipped entries has m_s = -inf and drops out).  One 128-thread block per (unit, head): the
-// first warp turns the ranges' (m, l) into weights in shared memory (splits <= 32), then each
-// thread accumulates 4 of the 512 output columns over the ranges.
+// skipped entries has m_s = -inf and drops out).  One 128-thread block per (unit, head, 128
+// output columns): every thread issues the loads of its column in all ranges (splits <= 32) at
+// once, the first warp meanwhile turns the ranges' (m, l) into weights in shared memory, and the
+// thread then sums its column.  Four blocks per head spread one query row's merge over the SMs.
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(128)
     latent_merge_kernel(const float* __restrict__ part, int HB, int hblocks, int splits, int Hq,
                         void* __restrict__ O) {
+    constexpr int CB = DV / 128;  // column blocks per head
     __shared__ float wt[32];
     __shared__ float inv_l;
-    const long long u = blockIdx.x / HB;  // (row, head block)
-    const int h = static_cast<int>(blockIdx.x % HB);
+    const long long uh = blockIdx.x / CB;  // (unit, head)
+    const int cb = static_cast<int>(blockIdx.x % CB);
+    const long long u = uh / HB;           // (row, head block)
+    const int h = static_cast<int>(uh % HB);
     const long long row = u / hblocks;
     const int hb = static_cast<int>(u % hblocks);
     const size_t sstride = static_cast<size_t>(HB) * (DV + 2);
     const float* p0 = part + (static_cast<size_t>(u) * splits * HB + h) * (DV + 2);
+    const int d = cb * 128 + threadIdx.x;
+    float v[32];
+#pragma unroll
+    for (int s2 = 0; s2 < 32; ++s2) v[s2] = s2 < splits ? __ldg(p0 + s2 * sstride + d) : 0.f;
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         const float m = lane < splits ? __ldg(p0 + lane * sstride + DV) : -INFINITY;
@@ -301,37 +309,24 @@ __global__ void __launch_bounds__(128)
         if (lane == 0) inv_l = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    const int d = threadIdx.x * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int s2 = 0; s2 < splits; ++s2) {
-        const float fs = wt[s2];
-        const float* src = p0 + s2 * sstride + d;
-        // rows of DV + 2 floats: 8-byte aligned, so two float2 loads
-        const float2 a = __ldg(reinterpret_cast<const float2*>(src));
-        const float2 c = __ldg(reinterpret_cast<const float2*>(src + 2));
-        acc.x += fs * a.x;
-        acc.y += fs * a.y;
-        acc.z += fs * c.x;
-        acc.w += fs * c.y;
-    }
-    const float inv = inv_l;
+    float acc = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 32; ++s2)
+        if (s2 < splits) acc = fmaf(wt[s2], v[s2], acc);
+    const float out = acc * inv_l;
     const size_t ob = (static_cast<size_t>(row) * Hq + static_cast<size_t>(hb) * HB + h) * DV + d;
-    if (OUT_BF16) {
-        __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(O) + ob;
-        *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-        *reinterpret_cast<__nv_bfloat162*>(op + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    } else {
-        float* op = reinterpret_cast<float*>(O) + ob;
-        *reinterpret_cast<float4*>(op) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    }
+    if (OUT_BF16)
+        reinterpret_cast<__nv_bfloat16*>(O)[ob] = __float2bfloat16_rn(out);
+    else
+        reinterpret_cast<float*>(O)[ob] = out;
 }
 
 }  // namespace lat
 
 cudaError_t launch_latent_merge(const float* part, int HB, int hblocks, int splits, long long units, int Hq, void* O,
                                 bool out_bf16, cudaStream_t stream) {
-    const unsigned mblocks = static_cast<unsigned>(units * HB);
+    if (splits > 32) return cudaErrorInvalidValue;  // one lane per range in the merge
+    const unsigned mblocks = static_cast<unsigned>(units * HB * (lat::DV / 128));
     if (out_bf16)
         lat::latent_merge_kernel<true><<<mblocks, 128, 0, stream>>>(part, HB, hblocks, splits, Hq, O);
     else
