@@ -127,8 +127,12 @@ __global__ void __launch_bounds__(WARPS * 32)
         const int sp = SPLIT ? static_cast<int>(it % splits) : 0;
         const int c0 = SPLIT ? sp * chunks_per_split : 0;
         const int c1 = SPLIT ? min(nchunks, c0 + chunks_per_split) : nchunks;
-        const long long row = u / Hkv;
-        const int g = static_cast<int>(u % Hkv);
+        // unsplit units run KV head by KV head (all rows of head 0, then head 1, ...): the rows in
+        // flight at once then gather from one head's K/V, which fits in L2 where all heads' do not;
+        // split ranges keep (row, head) order, the order their merge reads them in
+        const long long nrows = static_cast<long long>(B) * n_q;
+        const long long row = SPLIT ? u / Hkv : u % nrows;
+        const int g = static_cast<int>(SPLIT ? u % Hkv : u / nrows);
         const long long b = row / n_q;
         const int qi = static_cast<int>(row - b * n_q);
         const int* irow = SHARED ? idx + (b * share.rows(n_q) + qi / share.q_per_idx) * topk : idx + row * topk;
