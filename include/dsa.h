@@ -251,9 +251,10 @@ DSA_API int sparse_attn_topk_shared(const void* Q, const void* K, const void* V,
  *   idx_out    [B, topk] int32: logical token indices, ascending, then -1.
  * Requires H_I in {32, 64}, d_I = 128, page_size a power of two >= 16,
  * max_pages * page_size >= max_seq_len >= every seq_lens[b] >= 1 (a length
- * outside [1, max_pages * page_size] is flagged DSA_STATUS_BAD_INDEX and
- * clamped; page numbers outside [0, num_pages) read page 0, whose keys are
- * masked).  max_seq_len (host) sizes the work split.
+ * outside [1, max_seq_len] is flagged DSA_STATUS_BAD_INDEX and clamped; page
+ * numbers outside [0, num_pages) read page 0, whose keys are masked).
+ * max_seq_len (host) sizes the work split and the per-sequence score keys
+ * the selection reads (4 bytes per token of max_seq_len in the workspace).
  *
  * sparse_attn_topk_paged: attention of each sequence's query over its
  * selected tokens (logical indices, as idx_score_topk_paged writes them).

@@ -11,15 +11,16 @@
 //   * The MMA is 128 keys x H_I heads (N = H_I, one query) and the 512 TMEM
 //     columns hold a ring of 512/H_I accumulators, so many key tiles are in
 //     flight while the epilogue drains older ones.
-//   * A 4-stage TMA ring streams the keys; the candidate buffer of the unit's
-//     single row lives in shared memory.
-//   * Each unit writes its partial top-k (ascending indices with their score
-//     keys); topk_merge_pairs then selects the final top-k of each sequence
-//     from its units' lists (dsa_topk_scores.cu).
+//   * A TMA ring of 128 KB streams the keys (4 bf16 or 8 fp8 stages).
+//   * Each unit writes its keys' order-preserving score keys to the row's slots
+//     and counts their top bits into a histogram (in the shared memory a
+//     candidate buffer would take), added to the row's histogram from the
+//     unit's own k-th-key bin up; the bin select (dsa_topk_radix.cu) then
+//     picks each row's top-k in one pass over its score keys.
 //   * The key cache may be paged (serving: fixed-size pages of tokens, a page
 //     table per sequence) and sequences may differ in length: each 128-key
 //     tile is fetched page by page, keys past a sequence's length are masked,
-//     and units past a sequence's last tile select nothing.
+//     and units past a sequence's last tile score nothing.
 #include <cuda.h>
 
 #include "dsa_tc.cuh"
@@ -27,12 +28,10 @@
 
 namespace dsa {
 
-cudaError_t launch_topk_merge_pairs(const uint32_t* keys, const int* idxs, int rows, int len, int k, int* out,
-                                    WsHeader* hdr, int num_sms, cudaStream_t stream, int n_tok);
 size_t bin_topk_hist_bytes(int rows);
 size_t bin_topk_scratch_bytes(int rows, int n, int num_sms);
 cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
-                            WsHeader* hdr, int num_sms, cudaStream_t stream);
+                            WsHeader* hdr, const int* lens, int len_cap, int num_sms, cudaStream_t stream);
 
 template <int H, bool FP8>
 struct DecCfg {
@@ -70,8 +69,6 @@ struct DecParams {
     const int* page_table;  // [B, max_pages] physical page of each logical page, or NULL: contiguous [B, n_kv]
     int page_size, max_pages, num_pages;
     int B, q_pos0, n_kv, topk, splits, tiles_per_split;
-    uint32_t* part_key;  // [B * splits, topk]
-    int* part_idx;       // [B * splits, topk]
     uint32_t* score_keys;  // [B, q_pos0 + 1] order-preserving score keys (score mode), or NULL
     int* hist;             // score mode: [B, 2^kBinTopkBits] counts of the keys' top bits (zeroed before)
     WsHeader* hdr;
@@ -87,11 +84,9 @@ __global__ void __launch_bounds__(192, 1)
     unsigned char* sB = smem + C::OFF_B;
     unsigned char* sA = smem + C::OFF_A;
     uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + C::OFF_CK);
-    int* cidx = reinterpret_cast<int*>(smem + C::OFF_CI);
     int* sortbuf = reinterpret_cast<int*>(smem + C::OFF_SORT);
     float* ws = reinterpret_cast<float*>(smem + C::OFF_W);
     auto* sc = reinterpret_cast<TopkGroup<128>::Scratch*>(smem + C::OFF_SC);
-    TopkRowState* st = reinterpret_cast<TopkRowState*>(smem + C::OFF_ST);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars + 0;
     uint64_t* q_empty = bars + 1;
@@ -139,7 +134,8 @@ __global__ void __launch_bounds__(192, 1)
     auto seq_len = [&](int b) -> int {
         if (!p.seq_lens) return p.q_pos0 + 1;
         int len = __ldg(p.seq_lens + b);
-        const int cap = p.page_table ? p.max_pages * p.page_size : p.n_kv;
+        // at most the row of score keys (max_seq_len for a paged cache) and the pages it holds
+        const int cap = p.page_table ? min(p.max_pages * p.page_size, p.q_pos0 + 1) : p.n_kv;
         if (len < 1 || len > cap) {
             if (threadIdx.x == 0) raise_status(p.hdr, DSA_STATUS_BAD_INDEX, len);
             len = len < 1 ? 1 : cap;
@@ -249,10 +245,8 @@ __global__ void __launch_bounds__(192, 1)
     } else {
         // ================================================== epilogue (warps 0-3)
         const int tid = threadIdx.x;  // key lane
-        TopkGroup<128> grp{tid, 1, sc, C::CAP};
-        const int sub = grp.sub();
-        constexpr int CHECK = 4;
-        const int room = sub - CHECK * 32;
+        TopkGroup<128> grp{tid, 1, sc, C::CAP};  // its named barrier for the four epilogue warps
+        constexpr int CHECK = 4;                 // tiles between looks at the abort word
         const uint32_t tlane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         uint32_t ua = 0;
         bool ok = true;
@@ -264,15 +258,10 @@ __global__ void __launch_bounds__(192, 1)
                 if (FP8) wv *= p.q_scale[static_cast<size_t>(b) * H + tid];
                 ws[tid] = wv;
             }
-            if (tid == 0) topk_row_init(st);
-            // score mode: the unit's histogram of its keys' top bits lives where the candidates would
+            // the unit's histogram of its score keys' top bits lives where candidate buffers would
             int* shist = reinterpret_cast<int*>(ckey);  // 2^kBinTopkBits counts in the ckey + cidx region
-            if (p.score_keys)
-                for (int i = tid; i < (1 << kBinTopkBits); i += 128) shist[i] = 0;
+            for (int i = tid; i < (1 << kBinTopkBits); i += 128) shist[i] = 0;
             grp.sync();
-            int cnt = 0;
-            uint32_t* wkey = ckey + warp * sub;
-            int* widx = cidx + warp * sub;
             for (int j = j0; j < j1; ++j, ++ua) {
                 const int a = ua % C::NACC;
                 const int s_key = j * 128 + tid;
@@ -307,37 +296,22 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (FP8) sc_v *= ksc;
                 const uint32_t key = score_key(sc_v);
-                if (p.score_keys) {
-                    // score mode: the row's keys go to memory and into the histogram of their top bits;
-                    // the bin select picks the top-k
-                    const bool v = got && s_key < len;
-                    if (v) p.score_keys[static_cast<size_t>(b) * (p.q_pos0 + 1) + s_key] = key;
-                    if (v) atomicAdd(&shist[key >> (32 - kBinTopkBits)], 1);
-                } else {
-                    const uint32_t tk = st->thr_key;
-                    const bool adm = got & (s_key < len) & ((key > tk) | ((key == tk) & (s_key < st->thr_idx)));
-                    topk_append_warp(wkey, widx, cnt, key, s_key, adm, sub);
+                // the row's keys go to memory and into the histogram of their top bits; the bin
+                // select picks the top-k
+                const bool v = got && s_key < len;
+                if (v) {
+                    p.score_keys[static_cast<size_t>(b) * (p.q_pos0 + 1) + s_key] = key;
+                    atomicAdd(&shist[key >> (32 - kBinTopkBits)], 1);
                 }
                 if (((j - j0) % CHECK) == CHECK - 1 || j == j1 - 1) {
-                    if (lane == 0) st->cnt[warp] = cnt;
                     grp.sync();
-                    int mx = 0, tot = 0;
-#pragma unroll
-                    for (int ww = 0; ww < 4; ++ww) {
-                        mx = max(mx, st->cnt[ww]);
-                        tot += st->cnt[ww];
-                    }
                     const bool stop = *wg_abort != 0;  // read between two barriers: uniform
                     grp.sync();
                     if (stop) { ok = false; break; }
-                    if (mx > room && tot > p.topk) {
-                        grp.prune(st, ckey, cidx, p.topk, room - 32, sortbuf);
-                        cnt = st->cnt[warp];
-                    }
                 }
             }
             if (!ok) break;
-            if (p.score_keys) {
+            {
                 grp.sync();  // every key of the unit is counted
                 // Only the bins from this unit's own k-th key up go to the row's histogram: the unit
                 // alone holds k keys at or above that bin, so the row's k-th key lies there too, and
@@ -374,12 +348,7 @@ __global__ void __launch_bounds__(192, 1)
                     if (c) atomicAdd(gh + i, c);
                 }
                 grp.sync();  // before the next unit clears it
-                continue;
             }
-            if (lane == 0) st->cnt[warp] = cnt;
-            grp.sync();
-            grp.finish(st, ckey, cidx, p.topk, p.part_idx + static_cast<size_t>(u) * p.topk,
-                       p.part_key + static_cast<size_t>(u) * p.topk, sortbuf);
         }
     }
 
@@ -478,31 +447,22 @@ cudaError_t launch_dec_t(const void* q, const float* q_scale, const void* k, con
     p.splits = (nkt + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty units
     p.hdr = static_cast<WsHeader*>(ws);
     unsigned char* scratch = static_cast<unsigned char*>(ws) + kWsHeaderBytes;
-    const bool bins = !paged;  // contiguous caches: score keys and their histogram, then the bin select
-    const size_t parts = static_cast<size_t>(B) * p.splits * topk;
-    p.part_key = reinterpret_cast<uint32_t*>(scratch);
-    p.part_idx = reinterpret_cast<int*>(p.part_key + parts);
-    p.score_keys = nullptr;
-    p.hist = nullptr;
+    // every row's score keys (max_len of them per row) and their histogram, then the bin select
     const size_t keys_bytes = (static_cast<size_t>(B) * max_len * 4 + 255) / 256 * 256;
-    if (bins) {
-        p.part_key = nullptr;
-        p.part_idx = nullptr;
-        p.score_keys = reinterpret_cast<uint32_t*>(scratch);
-        p.hist = reinterpret_cast<int*>(scratch + keys_bytes);
-    }
+    p.score_keys = reinterpret_cast<uint32_t*>(scratch);
+    p.hist = reinterpret_cast<int*>(scratch + keys_bytes);
     auto kern = indexer_decode_kernel<H, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    if (bins && (e = cudaMemsetAsync(p.hist, 0, bin_topk_hist_bytes(B), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.hist, 0, bin_topk_hist_bytes(B), stream)) != cudaSuccess) return e;
     const int units = B * p.splits;
     kern<<<units < num_sms ? units : num_sms, C::THREADS, C::SMEM, stream>>>(mq, mk, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (bins)
-        return launch_bin_topk(p.score_keys, max_len, B, max_len, topk, idx_out, scratch + keys_bytes, p.hdr,
-                               num_sms, stream);
-    return launch_topk_merge_pairs(p.part_key, p.part_idx, B, p.splits * topk, topk, idx_out, p.hdr, num_sms,
-                                   stream, max_len);
+    // variable lengths: the select reads each row's length, clamped as the kernel clamped it
+    const int len_cap = paged ? (pc.max_pages * pc.page_size < max_len ? pc.max_pages * pc.page_size : max_len)
+                              : max_len;
+    return launch_bin_topk(p.score_keys, max_len, B, max_len, topk, idx_out, scratch + keys_bytes, p.hdr,
+                           pc.seq_lens, len_cap, num_sms, stream);
 }
 
 }  // namespace
@@ -516,15 +476,12 @@ bool indexer_decode_supported(int B, int n_q, int q_pos0, int n_kv, int H, int d
 }
 
 size_t indexer_decode_workspace_bytes(int B, int q_pos0, int topk, int num_sms, bool varlen) {
-    if (!varlen) {  // contiguous caches: the row's score keys, then the bin select's state
-        const size_t keys_bytes = (static_cast<size_t>(B) * (q_pos0 + 1) * 4 + 255) / 256 * 256;
-        return keys_bytes + bin_topk_scratch_bytes(B, q_pos0 + 1, num_sms);
-    }
-    const int nkt = (q_pos0 + 1 + 127) / 128;  // varlen: q_pos0 = the longest sequence - 1
-    int splits = dec_splits(B, nkt, num_sms, per_sm_for(B, varlen));
-    const int tps = (nkt + splits - 1) / splits;
-    splits = (nkt + tps - 1) / tps;
-    return static_cast<size_t>(B) * splits * topk * 8;
+    // the rows' score keys (q_pos0 + 1 per row; for variable lengths q_pos0 = the longest - 1),
+    // then the bin select's state
+    (void)topk;
+    (void)varlen;
+    const size_t keys_bytes = (static_cast<size_t>(B) * (q_pos0 + 1) * 4 + 255) / 256 * 256;
+    return keys_bytes + bin_topk_scratch_bytes(B, q_pos0 + 1, num_sms);
 }
 
 cudaError_t launch_indexer_decode(const void* q, const float* q_scale, const void* k, const float* k_scale,

@@ -113,14 +113,21 @@ __device__ int bs_threshold_bin(const int* __restrict__ h, int k, int* hs, int* 
     return T;
 }
 
+// Keys in row `row`: n, or its own length clamped to [1, cap] when the rows differ.
+__device__ __forceinline__ int bs_row_len(int n, const int* lens, int cap, int row) {
+    if (!lens) return n;
+    const int len = __ldg(lens + row);
+    return len < 1 ? 1 : (len > cap ? cap : len);
+}
+
 // Keys of one slice with bin >= T, in token order, into the slice's region; the slice's count
 // (uncapped: a count above kBsSliceCap marks the row for the whole-row select).  Each thread
 // takes 8 consecutive keys of a 2048-key chunk, a block scan orders the kept keys, and a running
 // base carries across chunks.
 __global__ void __launch_bounds__(kRxThreads)
-    bin_compact_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int per, int k,
-                       const int* __restrict__ hist, uint32_t* __restrict__ ckey, int* __restrict__ cidx,
-                       int* __restrict__ ccnt) {
+    bin_compact_kernel(const uint32_t* __restrict__ keys, long long ld, int n, const int* __restrict__ lens,
+                       int len_cap, int nblk, int per, int k, const int* __restrict__ hist,
+                       uint32_t* __restrict__ ckey, int* __restrict__ cidx, int* __restrict__ ccnt) {
     __shared__ int2 wt[kRxThreads / 32];
     __shared__ int tsum[kRxThreads / 32];
     __shared__ int res;
@@ -129,7 +136,8 @@ __global__ void __launch_bounds__(kRxThreads)
     const uint32_t T = static_cast<uint32_t>(
         bs_threshold_bin(hist + static_cast<size_t>(row) * kBsBins, k, hs, tsum, &res));
     const uint32_t* kr = keys + row * ld;
-    const int i0 = blk * per, i1 = min(n, i0 + per);
+    const int nr = bs_row_len(n, lens, len_cap, row);
+    const int i0 = blk * per, i1 = min(nr, i0 + per);
     uint32_t* ok = ckey + static_cast<size_t>(blockIdx.x) * kBsSliceCap;
     int* oi = cidx + static_cast<size_t>(blockIdx.x) * kBsSliceCap;
     int base = 0;
@@ -271,9 +279,9 @@ __device__ void bs_write(KeyAt key_at, IdxAt idx_at, int m, int k, uint32_t K, i
 }
 
 __global__ void __launch_bounds__(kBsThreads)
-    bin_final_kernel(const uint32_t* __restrict__ keys, long long ld, int n, int nblk, int k,
-                     const uint32_t* __restrict__ ckey, const int* __restrict__ cidx, const int* __restrict__ ccnt,
-                     int* __restrict__ out, WsHeader* hdr) {
+    bin_final_kernel(const uint32_t* __restrict__ keys, long long ld, int n, const int* __restrict__ lens,
+                     int len_cap, int nblk, int k, const uint32_t* __restrict__ ckey, const int* __restrict__ cidx,
+                     const int* __restrict__ ccnt, int* __restrict__ out, WsHeader* hdr) {
     extern __shared__ __align__(16) unsigned char bs_smem[];
     uint32_t* skey = reinterpret_cast<uint32_t*>(bs_smem);
     int* sidx = reinterpret_cast<int*>(skey + kBsSmemCand);
@@ -339,10 +347,11 @@ __global__ void __launch_bounds__(kBsThreads)
         if (threadIdx.x == 0 && hdr) atomicMax(&hdr->sel_max_kept, total);
     } else {
         // the kept keys do not fit: select from the whole row
+        const int nr = bs_row_len(n, lens, len_cap, row);
         auto key_at = [&](int i) { return __ldg(kr + i); };
         auto idx_at = [&](int i) { return i; };
-        bs_kth(key_at, n, k, sh, sel, &K, &kk);
-        bs_write(key_at, idx_at, n, k, K, kk, wtot, orow);
+        bs_kth(key_at, nr, k, sh, sel, &K, &kk);
+        bs_write(key_at, idx_at, nr, k, K, kk, wtot, orow);
         if (threadIdx.x == 0 && hdr) atomicAdd(&hdr->sel_full_rows, 1);
     }
 }
@@ -371,10 +380,11 @@ size_t bin_topk_scratch_bytes(int rows, int n, int num_sms) {
     return bin_topk_hist_bytes(rows) + nb * sizeof(int) + nb * kBsSliceCap * (sizeof(uint32_t) + sizeof(int));
 }
 
-// Top-k of `rows` rows of n keys (row stride ld) whose histograms of the top kBsBits bits are at
-// the start of `scratch` -> out [rows, k] ascending tokens, then -1.
+// Top-k of `rows` rows of n keys (row stride ld; with `lens`, row r holds its own length clamped
+// to [1, len_cap]) whose histograms of the top kBsBits bits are at the start of `scratch`
+// -> out [rows, k] ascending tokens, then -1.
 cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n, int k, int* out, void* scratch,
-                            WsHeader* hdr, int num_sms, cudaStream_t stream) {
+                            WsHeader* hdr, const int* lens, int len_cap, int num_sms, cudaStream_t stream) {
     int per = 0;
     const int nblk = radix_blocks(rows, n, num_sms, &per);
     int* hist = static_cast<int*>(scratch);
@@ -385,9 +395,10 @@ cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n,
     cudaError_t e = cudaFuncSetAttribute(bin_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(fsm));
     if (e != cudaSuccess) return e;
-    bin_compact_kernel<<<static_cast<unsigned>(rows) * nblk, kRxThreads, 0, stream>>>(keys, ld, n, nblk, per, k, hist,
-                                                                                       ckey, cidx, ccnt);
-    bin_final_kernel<<<rows, kBsThreads, fsm, stream>>>(keys, ld, n, nblk, k, ckey, cidx, ccnt, out, hdr);
+    bin_compact_kernel<<<static_cast<unsigned>(rows) * nblk, kRxThreads, 0, stream>>>(
+        keys, ld, n, lens, len_cap, nblk, per, k, hist, ckey, cidx, ccnt);
+    bin_final_kernel<<<rows, kBsThreads, fsm, stream>>>(keys, ld, n, lens, len_cap, nblk, k, ckey, cidx, ccnt, out,
+                                                        hdr);
     return cudaGetLastError();
 }
 

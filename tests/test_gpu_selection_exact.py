@@ -6,9 +6,9 @@ equal the oracle's bit for bit, and the selection rule (k largest, ties to the l
 index, ascending output, -1 padding) leaves exactly one correct answer.  Small value
 ranges make equal scores and zero scores common, so tie-breaking, the streaming prune of
 the fused kernel (and its exact fallback when one score value holds more ties than the
-prune's slack), the split decode kernel's partial lists and both of its merges are all
-checked for exactness, not within a tolerance; so is the bin select (histogram of the score
-keys' top bits, kept keys, exact select) that one-query decode over a contiguous cache uses.
+prune's slack) and the bin select of one-query decode (histogram of the score keys' top
+bits, kept keys, exact select; whole-row select when the kept keys overflow), over
+contiguous and paged caches, are all checked for exactness, not within a tolerance.
 
 [QbitAI] §IndexCache / [Term] "dot product + top-k": the selection is the k best scores
 of each query row; ties to the lower index is this library's stated rule.
@@ -128,7 +128,7 @@ def _decode_case(name, B, n_kv, H, topk, lo, hi, fp8=False):
 
 
 @pytest.mark.parametrize("case", [
-    # (name, B, n_kv, H, topk, lo, hi): the bitmap merge of the split lists
+    # (name, B, n_kv, H, topk, lo, hi): one query per sequence, the bin select
     ("dec_b4_h32", 4, 20000, 32, 2048, -4, 4),
     ("dec_b2_h64_ties", 2, 9000, 64, 2048, -1, 1),
     ("dec_b8_h32_k300", 8, 4100, 32, 300, -3, 3),
@@ -177,9 +177,9 @@ def test_decode_bin_select_fast_path_and_whole_row_fallback_are_exact():
     assert full == 2, (full, kept)
 
 
-def test_paged_decode_streaming_merge_selection_is_exact():
-    """A paged sequence of 1.7M tokens: the position bitmap of the split merge would not fit in
-    shared memory, so the split lists go through the streaming merge."""
+def test_paged_decode_long_sequence_selection_is_exact():
+    """A paged sequence of 1.7M tokens in shuffled pages: its score keys and histogram, then the
+    bin select (with these heavily tied scores, its whole-row select)."""
     n, P, H, d, topk = 1_700_000, 256, 32, 128, 2048
     q, k, w = synth.integer_indexer("paged_stream", 1, n, H, d, -2, 2, q_rows=1)
     pages = (n + P - 1) // P
