@@ -104,9 +104,8 @@ extern "C" DSA_API int idx_score_topk_noalloc(const void* q_I, const float* q_sc
     const size_t fit = room / per_cta;
     int max_ctas = static_cast<int>(fit < static_cast<size_t>(sms) ? fit : static_cast<size_t>(sms));
     // The estimate above is exact for the prefill kernel, whose scratch grows with its grid.  The
-    // one-query decode kernel sizes its partial lists by a split count that is a step function of
-    // the SM count it is given, so check the bytes the launch will really use and shrink the grid
-    // until they fit.
+    // one-query decode route sizes its selection scratch (slices per row) by the SM count it is
+    // given, so check the bytes the launch will really use and shrink the grid until they fit.
     while (max_ctas > 1 &&
            dsa::indexer_workspace_bytes(B, n_q, q_pos0, n_kv, H_I, d_I, topk, dtype, max_ctas) > room)
         --max_ctas;
