@@ -88,6 +88,15 @@ def test_paged_decode_flags_bad_lengths_and_indices():
     ws = torch.zeros(dsa.idx_score_topk_paged_workspace_size(2, 300, H, d, k), dtype=torch.uint8, device=DEV)
     dsa.idx_score_topk_paged(bt["q"].to(DEV), k_pages, table, bad_len, bt["w"].to(DEV), k, 300, workspace=ws)
     assert dsa.read_status(ws) & dsa.STATUS_BAD_INDEX
+    # a length above max_seq_len (here still within the sequence's pages) is flagged and clamped
+    # to max_seq_len: the per-sequence score slots hold max_seq_len keys
+    assert bt["table"].shape[1] * P > 350
+    ws.zero_()
+    long_len = torch.tensor([350, 200], dtype=torch.int32, device=DEV)
+    out = dsa.idx_score_topk_paged(bt["q"].to(DEV), k_pages, table, long_len, bt["w"].to(DEV), k, 300,
+                                   workspace=ws)
+    assert dsa.read_status(ws) & dsa.STATUS_BAD_INDEX
+    assert int(out.max()) < 300
     # an index at or beyond its sequence's length is skipped and flagged
     seq = torch.from_numpy(bt["lens"]).to(DEV)
     idx = torch.full((2, k), -1, dtype=torch.int32)
