@@ -66,9 +66,10 @@ constexpr int kBsThreads = 512;
 constexpr int kBsSliceCap = 2048;
 constexpr int kBsSmemCand = 16384;
 
-// The largest bin T with count(bins >= T) >= k in one row's histogram (0 when the row holds k
-// keys or fewer: everything is kept); every thread of the kRxThreads-thread block gets it.
-__device__ int bs_threshold_bin(const int* __restrict__ h, int k, int* hs, int* tsum, int* res) {
+// The largest bin T with count(bins >= T) >= k in one row's histogram, and the count of keys in
+// the bins above it (T = 0, above = -1 when the row holds fewer than k keys: everything is kept);
+// every thread of the kRxThreads-thread block gets them.
+__device__ int bs_threshold_bin(const int* __restrict__ h, int k, int* hs, int* tsum, int* res, int* above_out) {
     constexpr int PB = kBsBins / kRxThreads;  // bins per thread
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     // the histogram into shared memory with coalesced 16-byte loads, then contiguous ranges per thread
@@ -90,7 +91,10 @@ __device__ int bs_threshold_bin(const int* __restrict__ h, int k, int* hs, int* 
         if (lane + off < 32) suf += o;
     }
     if (lane == 0) tsum[w] = suf;  // this warp's total
-    if (t == 0) *res = 0;
+    if (t == 0) {
+        res[0] = 0;
+        res[1] = -1;
+    }
     __syncthreads();
     int later = 0;  // keys in the warps above this one
     for (int j = w + 1; j < kRxThreads / 32; ++j) later += tsum[j];
@@ -99,16 +103,19 @@ __device__ int bs_threshold_bin(const int* __restrict__ h, int k, int* hs, int* 
     if (suf >= k && above_me < k) {
         int acc = above_me, T = t * PB;
         for (int j = PB - 1; j >= 0; --j) {
-            acc += hs[t * PB + j];
-            if (acc >= k) {
+            const int c = hs[t * PB + j];
+            if (acc + c >= k) {
                 T = t * PB + j;
                 break;
             }
+            acc += c;
         }
-        *res = T;
+        res[0] = T;
+        res[1] = acc;  // keys in bins above T
     }
     __syncthreads();
-    const int T = *res;
+    const int T = res[0];
+    *above_out = res[1];
     __syncthreads();
     return T;
 }
@@ -127,23 +134,19 @@ __device__ __forceinline__ int bs_row_len(int n, const int* lens, int cap, int r
 __global__ void __launch_bounds__(kRxThreads)
     bin_compact_kernel(const uint32_t* __restrict__ keys, long long ld, int n, const int* __restrict__ lens,
                        int len_cap, int nblk, int per, int k, const int* __restrict__ hist,
-                       uint32_t* __restrict__ ckey, int* __restrict__ cidx, int* __restrict__ ccnt) {
+                       uint32_t* __restrict__ ckey, int* __restrict__ cidx, int* __restrict__ ccnt,
+                       int2* __restrict__ rinfo) {
     __shared__ int2 wt[kRxThreads / 32];
     __shared__ int tsum[kRxThreads / 32];
-    __shared__ int res;
+    __shared__ int res[2];
     __shared__ __align__(16) int hs[kBsBins];
     const int row = blockIdx.x / nblk, blk = blockIdx.x % nblk;
-    const uint32_t T = static_cast<uint32_t>(
-        bs_threshold_bin(hist + static_cast<size_t>(row) * kBsBins, k, hs, tsum, &res));
     const uint32_t* kr = keys + row * ld;
     const int nr = bs_row_len(n, lens, len_cap, row);
     const int i0 = blk * per, i1 = min(nr, i0 + per);
-    uint32_t* ok = ckey + static_cast<size_t>(blockIdx.x) * kBsSliceCap;
-    int* oi = cidx + static_cast<size_t>(blockIdx.x) * kBsSliceCap;
-    int base = 0;
-    for (int c0 = i0; c0 < i1; c0 += kRxThreads * 8) {
+    // 8 consecutive keys of the chunk at c0 for this thread (two 16-byte loads when aligned)
+    auto load8 = [&](int c0, uint32_t (&kv)[8]) {
         const int a = c0 + threadIdx.x * 8;
-        uint32_t kv[8];
         if (a + 8 <= i1 && ((row * ld + a) & 3) == 0) {
             const uint4 x = __ldg(reinterpret_cast<const uint4*>(kr + a));
             const uint4 y = __ldg(reinterpret_cast<const uint4*>(kr + a + 4));
@@ -153,6 +156,22 @@ __global__ void __launch_bounds__(kRxThreads)
 #pragma unroll
             for (int e = 0; e < 8; ++e) kv[e] = a + e < i1 ? __ldg(kr + a + e) : 0u;
         }
+    };
+    uint32_t nx[8];
+    load8(i0, nx);  // the first chunk's keys load while the threshold is found
+    int above;
+    const uint32_t T = static_cast<uint32_t>(
+        bs_threshold_bin(hist + static_cast<size_t>(row) * kBsBins, k, hs, tsum, res, &above));
+    if (blk == 0 && threadIdx.x == 0) rinfo[row] = make_int2(static_cast<int>(T), above);
+    uint32_t* ok = ckey + static_cast<size_t>(blockIdx.x) * kBsSliceCap;
+    int* oi = cidx + static_cast<size_t>(blockIdx.x) * kBsSliceCap;
+    int base = 0;
+    for (int c0 = i0; c0 < i1; c0 += kRxThreads * 8) {
+        const int a = c0 + threadIdx.x * 8;
+        uint32_t kv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kv[e] = nx[e];
+        if (c0 + kRxThreads * 8 < i1) load8(c0 + kRxThreads * 8, nx);  // the next chunk loads during this one
         int mine = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) mine += (a + e < i1) && (kv[e] >> kBsShift) >= T;
@@ -196,15 +215,18 @@ __device__ __forceinline__ int bs_excl_scan(int v, int* warp_tot, int* total) {
     return before + inc - v;
 }
 
-// The k-th largest of m keys produced by key_at(i) (i < m), and how many of the keys equal to it
-// are selected; 4 passes of 8 bits with a shared-memory histogram.
+// The need-th largest of the keys produced by key_at(i) (i < m) whose bits from lo_bit up equal
+// `prefix`, and how many of the keys equal to it are selected; passes of up to 8 bits from bit
+// lo_bit - 1 down, each with a shared-memory histogram.  (lo_bit = 32, prefix = 0: all m keys.)
 template <class KeyAt>
-__device__ void bs_kth(KeyAt key_at, int m, int k, int* sh, int* sel, uint32_t* K_out, int* kk_out) {
-    uint32_t prefix = 0u;
-    int need = min(k, m);
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        const uint32_t fixed = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+__device__ void bs_kth(KeyAt key_at, int m, int need, uint32_t prefix, int lo_bit, int* sh, int* sel,
+                       uint32_t* K_out, int* kk_out) {
+    while (lo_bit > 0) {
+        const int width = lo_bit < 8 ? lo_bit : 8;
+        const int shift = lo_bit - width;
+        const uint32_t fixed = lo_bit >= 32 ? 0u : (0xffffffffu << lo_bit);
+        const uint32_t dmask = (1u << width) - 1u;
+        lo_bit = shift;
         for (int b = threadIdx.x; b < 256; b += kBsThreads) sh[b] = 0;
         __syncthreads();
         // the keys share their top bits, so most lanes of a warp hit the same bin: one shared
@@ -215,7 +237,7 @@ __device__ void bs_kth(KeyAt key_at, int m, int k, int* sh, int* sel, uint32_t* 
             const bool in = i < m && (key & fixed) == prefix;
             const unsigned act = __ballot_sync(0xffffffffu, in);
             if (in) {
-                const uint32_t dg = (key >> shift) & 255u;
+                const uint32_t dg = (key >> shift) & dmask;
                 const unsigned same = __match_any_sync(act, dg);
                 if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sh[dg], __popc(same));
             }
@@ -281,7 +303,8 @@ __device__ void bs_write(KeyAt key_at, IdxAt idx_at, int m, int k, uint32_t K, i
 __global__ void __launch_bounds__(kBsThreads)
     bin_final_kernel(const uint32_t* __restrict__ keys, long long ld, int n, const int* __restrict__ lens,
                      int len_cap, int nblk, int k, const uint32_t* __restrict__ ckey, const int* __restrict__ cidx,
-                     const int* __restrict__ ccnt, int* __restrict__ out, WsHeader* hdr) {
+                     const int* __restrict__ ccnt, const int2* __restrict__ rinfo, int* __restrict__ out,
+                     WsHeader* hdr) {
     extern __shared__ __align__(16) unsigned char bs_smem[];
     uint32_t* skey = reinterpret_cast<uint32_t*>(bs_smem);
     int* sidx = reinterpret_cast<int*>(skey + kBsSmemCand);
@@ -342,7 +365,13 @@ __global__ void __launch_bounds__(kBsThreads)
         __syncthreads();
         auto key_at = [&](int i) { return skey[i]; };
         auto idx_at = [&](int i) { return sidx[i]; };
-        bs_kth(key_at, total, k, sh, sel, &K, &kk);
+        // the k-th key lies in bin T, below `above` keys of the higher bins: only bin T's keys and
+        // their low bits are left to search (every key is kept when the row holds fewer than k)
+        const int2 ri = rinfo[row];
+        if (ri.y < 0)
+            bs_kth(key_at, total, min(k, total), 0u, 32, sh, sel, &K, &kk);
+        else
+            bs_kth(key_at, total, k - ri.y, static_cast<uint32_t>(ri.x) << kBsShift, kBsShift, sh, sel, &K, &kk);
         bs_write(key_at, idx_at, total, k, K, kk, wtot, orow);
         if (threadIdx.x == 0 && hdr) atomicMax(&hdr->sel_max_kept, total);
     } else {
@@ -350,7 +379,7 @@ __global__ void __launch_bounds__(kBsThreads)
         const int nr = bs_row_len(n, lens, len_cap, row);
         auto key_at = [&](int i) { return __ldg(kr + i); };
         auto idx_at = [&](int i) { return i; };
-        bs_kth(key_at, nr, k, sh, sel, &K, &kk);
+        bs_kth(key_at, nr, min(k, nr), 0u, 32, sh, sel, &K, &kk);
         bs_write(key_at, idx_at, nr, k, K, kk, wtot, orow);
         if (threadIdx.x == 0 && hdr) atomicAdd(&hdr->sel_full_rows, 1);
     }
@@ -377,7 +406,8 @@ size_t bin_topk_hist_bytes(int rows) { return static_cast<size_t>(rows) * kBsBin
 size_t bin_topk_scratch_bytes(int rows, int n, int num_sms) {
     int per = 0;
     const size_t nb = static_cast<size_t>(rows) * radix_blocks(rows, n, num_sms, &per);
-    return bin_topk_hist_bytes(rows) + nb * sizeof(int) + nb * kBsSliceCap * (sizeof(uint32_t) + sizeof(int));
+    return bin_topk_hist_bytes(rows) + nb * sizeof(int) + nb * kBsSliceCap * (sizeof(uint32_t) + sizeof(int)) +
+           static_cast<size_t>(rows) * sizeof(int2);
 }
 
 // Top-k of `rows` rows of n keys (row stride ld; with `lens`, row r holds its own length clamped
@@ -387,8 +417,11 @@ cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n,
                             WsHeader* hdr, const int* lens, int len_cap, int num_sms, cudaStream_t stream) {
     int per = 0;
     const int nblk = radix_blocks(rows, n, num_sms, &per);
+    // hist | rinfo (8-byte records: right after the histograms, whose size is a multiple of 8) |
+    // ccnt | ckey | cidx
     int* hist = static_cast<int*>(scratch);
-    int* ccnt = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(scratch) + bin_topk_hist_bytes(rows));
+    int2* rinfo = reinterpret_cast<int2*>(reinterpret_cast<unsigned char*>(scratch) + bin_topk_hist_bytes(rows));
+    int* ccnt = reinterpret_cast<int*>(rinfo + rows);
     uint32_t* ckey = reinterpret_cast<uint32_t*>(ccnt + static_cast<size_t>(rows) * nblk);
     int* cidx = reinterpret_cast<int*>(ckey + static_cast<size_t>(rows) * nblk * kBsSliceCap);
     const size_t fsm = static_cast<size_t>(2 * kBsSmemCand + nblk + 1) * sizeof(int);
@@ -396,9 +429,9 @@ cudaError_t launch_bin_topk(const uint32_t* keys, long long ld, int rows, int n,
                                          static_cast<int>(fsm));
     if (e != cudaSuccess) return e;
     bin_compact_kernel<<<static_cast<unsigned>(rows) * nblk, kRxThreads, 0, stream>>>(
-        keys, ld, n, lens, len_cap, nblk, per, k, hist, ckey, cidx, ccnt);
-    bin_final_kernel<<<rows, kBsThreads, fsm, stream>>>(keys, ld, n, lens, len_cap, nblk, k, ckey, cidx, ccnt, out,
-                                                        hdr);
+        keys, ld, n, lens, len_cap, nblk, per, k, hist, ckey, cidx, ccnt, rinfo);
+    bin_final_kernel<<<rows, kBsThreads, fsm, stream>>>(keys, ld, n, lens, len_cap, nblk, k, ckey, cidx, ccnt, rinfo,
+                                                        out, hdr);
     return cudaGetLastError();
 }
 
