@@ -7,8 +7,9 @@
 // the keys' top bits into a histogram per row.  The selection then needs one pass over the keys:
 //   * compaction: each slice CTA finds the histogram bin that holds its row's k-th key and keeps
 //     its keys from that bin up, in token order (fewer than k above the bin, plus the bin);
-//   * final: one CTA per row selects among the kept keys in shared memory (radix select of the
-//     exact k-th key, equal keys taken in token order) and writes the tokens in order.
+//   * final: one CTA per row selects among the kept keys in shared memory (the exact k-th key is
+//     searched among the keys of its bin alone, equal keys taken in token order) and writes the
+//     tokens in order.
 // A row whose kept keys do not fit (scores packed into one bin, many equal scores) is selected by
 // the same CTA from its whole row.  No CTA ever waits for another: the steps are separate launches.
 #include "dsa_common.cuh"
@@ -55,8 +56,10 @@ __device__ __forceinline__ int2 block_excl_scan2(int2 v, int2* warp_tot, int2* t
 //     histogram (suffix counts), then keeps its keys whose bin is >= T, in token order, in its own
 //     region (at most kBsSliceCap) -- fewer than k keys above T plus the keys of bin T.
 //   * final: one CTA per row loads the row's kept keys (at most kBsSmemCand) into shared memory in
-//     token order, finds the k-th key K and how many keys equal to K to take by a radix select in
-//     shared memory, and writes the selected tokens in order.  A row whose kept keys overflow
+//     token order.  The compaction recorded T and the number of keys above it, so the k-th key K
+//     is the (k - above)-th largest key of bin T: a radix select over those keys' low
+//     32 - kBsBits bits finds it and how many keys equal to K to take.  The CTA then writes the
+//     selected tokens in order.  A row whose kept keys overflow
 //     either bound (a score distribution packed into a few bins, many equal scores) is selected
 //     by the same CTA directly from the full row instead.
 constexpr int kBsBits = kBinTopkBits;
