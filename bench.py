@@ -335,11 +335,11 @@ def run_gpu(args, rank, world, local_rank):
             "gathered_frac_equiv": round(abytes / (attn_avg / 1e3) / 1e9 / hbm, 4),
             "gathered_note": "algorithmic gathered bytes (sum_t min(k,t+1) x Hkv x 2d x 2 B) / launch time: above "
                              "HBM peak because every token is gathered by many queries and L2 serves the repeats "
-                             "(DRAM moves ~3 % of the gathered bytes); the kernel is bound by issue and by the L2-to-SM "
-                             "gather path, not by DRAM: a pure 16-byte cp.async copy through the same per-warp "
-                             "rings, with the same 2048-key units in the same KV-head order, moves 13.5 TB/s of "
-                             "uniform random rows of a 200K-token pool on this GPU (19.6 TB/s from a 16K-token "
-                             "pool that stays in L2)"},
+                             "(DRAM moves ~3 % of the gathered bytes); the kernel is bound by instruction issue and "
+                             "latency (57 % of issue slots used), not by DRAM or by the gather path: a pure "
+                             "16-byte cp.async copy through the same per-warp rings, with the same 2048-key units "
+                             "in the same KV-head order and ascending index lists, moves 19.1 TB/s of random rows "
+                             "of a 200K-token pool on this GPU"},
         "attention_random_indices": {
             "kernel": "sparse_attn_kernel, same shape and launch configuration, stratified random top-2048 rows",
             "avg_launch_ms": round(rnd_ms, 3),
