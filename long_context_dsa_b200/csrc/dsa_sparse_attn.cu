@@ -26,6 +26,7 @@
 //     (16-key chunks, 2 stages each) fit in shared memory at d = 128.  On
 //     B200 the number of warps in flight set the speed far more than the
 //     stages per warp did.
+#include <climits>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -90,9 +91,10 @@ struct AttnCfg {
 
 // Compile-time switches, so the plain path carries none of the bookkeeping of the others:
 // SPLIT: units cut into index ranges (few rows, e.g. decode); PAGED: K/V in a page pool;
-// SHARED: query rows share index rows.
+// SHARED: query rows share index rows; OFF32: every row of a sequence's K (and V) lies within
+// 2 GB of its first, so row offsets are 32-bit (contiguous caches only).
 template <int D, int CHUNK, int STAGES, int WARPS, bool SWZ, bool QK_SPLIT, bool OUT_BF16, bool SPLIT, bool PAGED,
-          bool SHARED>
+          bool SHARED, bool OFF32 = false>
 __global__ void __launch_bounds__(WARPS * 32)
     sparse_attn_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                        const __nv_bfloat16* __restrict__ V, const int* __restrict__ idx, int B, int n_q,
@@ -141,6 +143,9 @@ __global__ void __launch_bounds__(WARPS * 32)
         const __nv_bfloat16* kb = K + seq_off + static_cast<size_t>(g) * D;
         const __nv_bfloat16* vb = V + seq_off + static_cast<size_t>(g) * D;
         const int n_valid = PAGED ? min(__ldg(pg.lens + b), pg.max_pages * pg.page_size) : n_kv;
+        // OFF32: this lane's 16-byte segment of a row at byte offset 0 (K and V)
+        const unsigned char* kseg = reinterpret_cast<const unsigned char*>(kb) + seg * 16;
+        const unsigned char* vseg = reinterpret_cast<const unsigned char*>(vb) + seg * 16;
 
         // Index of key `lane` of chunk c (-1 past the end), read two chunks ahead of its gather, then
         // checked and mapped to its cache row one chunk ahead (so a page-table read never waits on
@@ -173,14 +178,29 @@ __global__ void __launch_bounds__(WARPS * 32)
                 if (lane < CHUNK) sidx[s * CHUNK + lane] = tsel;
                 const uint32_t kst = ring_s + s * C::STAGE_BYTES;
                 const uint32_t vst = kst + CHUNK * C::RS;
+                if constexpr (OFF32) {
+                    // the lane holding a key turns it into its row's byte offset once (padding: the
+                    // sign bit alone); the copying lanes shuffle that word in and mask it
+                    const int w = tsel >= 0 ? tsel * static_cast<int>(tok_stride * 2) : INT_MIN;
 #pragma unroll
-                for (int i = 0; i < CHUNK / C::KEYS_PER_INSN; ++i) {
-                    const int key = i * C::KEYS_PER_INSN + sub;
-                    const int t = __shfl_sync(0xffffffffu, tsel, key);
-                    const uint32_t nb = t >= 0 ? 16u : 0u;
-                    const size_t off = static_cast<size_t>(t >= 0 ? t : 0) * tok_stride + seg * 8;
-                    cp_async16(kst + C::at(key, seg), kb + off, nb);
-                    cp_async16(vst + C::at(key, seg), vb + off, nb);
+                    for (int i = 0; i < CHUNK / C::KEYS_PER_INSN; ++i) {
+                        const int key = i * C::KEYS_PER_INSN + sub;
+                        const int wk = __shfl_sync(0xffffffffu, w, key);
+                        const uint32_t nb = wk >= 0 ? 16u : 0u;
+                        const uint32_t o = static_cast<uint32_t>(wk) & 0x7fffffffu;
+                        cp_async16(kst + C::at(key, seg), kseg + o, nb);
+                        cp_async16(vst + C::at(key, seg), vseg + o, nb);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < CHUNK / C::KEYS_PER_INSN; ++i) {
+                        const int key = i * C::KEYS_PER_INSN + sub;
+                        const int t = __shfl_sync(0xffffffffu, tsel, key);
+                        const uint32_t nb = t >= 0 ? 16u : 0u;
+                        const size_t off = static_cast<size_t>(t >= 0 ? t : 0) * tok_stride + seg * 8;
+                        cp_async16(kst + C::at(key, seg), kb + off, nb);
+                        cp_async16(vst + C::at(key, seg), vb + off, nb);
+                    }
                 }
             }
             cp_async_commit();
@@ -475,9 +495,15 @@ static cudaError_t launch_attn_t(const __nv_bfloat16* Q, const __nv_bfloat16* K,
          {DSA_K(false, true, false, false), DSA_K(false, true, true, false), DSA_K(false, true, false, true)}},
         {{DSA_K(true, false, false, false), DSA_K(true, false, true, false), DSA_K(true, false, false, true)},
          {DSA_K(true, true, false, false), DSA_K(true, true, true, false), DSA_K(true, true, false, true)}}};
+#define DSA_K32(OB, SP) sparse_attn_kernel<D, CHUNK, STAGES, WARPS, SWZ, QK_SPLIT, OB, SP, false, false, true>
+    static const KernFn table32[2][2] = {{DSA_K32(false, false), DSA_K32(false, true)},
+                                         {DSA_K32(true, false), DSA_K32(true, true)}};
+#undef DSA_K32
 #undef DSA_K
     const int mode = pg.table ? 1 : (share.q_per_idx > 1 || share.causal) ? 2 : 0;
-    KernFn kern = table[out_bf16 ? 1 : 0][splits > 1 ? 1 : 0][mode];
+    // contiguous caches whose per-sequence K (and V) spans under 2 GB take 32-bit row offsets
+    const bool off32 = mode == 0 && static_cast<long long>(n_kv) * Hkv * D * 2 <= 0x7fffffffLL;
+    KernFn kern = off32 ? table32[out_bf16 ? 1 : 0][splits > 1 ? 1 : 0] : table[out_bf16 ? 1 : 0][splits > 1 ? 1 : 0][mode];
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
     if (e != cudaSuccess) return e;
     int per_sm = 0;
