@@ -26,6 +26,7 @@
 //     (16-key chunks, 2 stages each) fit in shared memory at d = 128.  On
 //     B200 the number of warps in flight set the speed far more than the
 //     stages per warp did.
+#include <cfloat>
 #include <climits>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(WARPS * 32)
         // gather chunk c's K and V slices into stage c % STAGES (always commits one group)
         auto issue = [&](int c, int tsel) {
             if (c < c1) {
-                const int s = (SPLIT ? c - c0 : c) % STAGES;
+                const int s = static_cast<int>(static_cast<unsigned>(SPLIT ? c - c0 : c) % STAGES);
                 if (lane < CHUNK) sidx[s * CHUNK + lane] = tsel;
                 const uint32_t kst = ring_s + s * C::STAGE_BYTES;
                 const uint32_t vst = kst + CHUNK * C::RS;
@@ -220,7 +221,11 @@ __global__ void __launch_bounds__(WARPS * 32)
         float o[D / 16][4];
 #pragma unroll
         for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-        float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
+        // running max starts at -FLT_MAX, not -inf: it stays finite, so the rescale and the weights
+        // need no guard (a masked score is -inf and weighs exp2(-inf) = 0; before any valid key
+        // the factor is exp2(0) = 1), and a range that saw no key reports -FLT_MAX to the merge,
+        // where it weighs 0 beside any range that did
+        float mrun[2] = {-FLT_MAX, -FLT_MAX}, lrun[2] = {0.f, 0.f};
 
         // prologue: stages 0 .. STAGES-2 in flight, the next chunk's rows and the one after's
         // indices in registers
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(WARPS * 32)
             r_next = load_raw(c + STAGES + 1);
             cp_async_wait<STAGES - 1>();
             __syncwarp();
-            const int s = (SPLIT ? c - c0 : c) % STAGES;
+            const int s = static_cast<int>(static_cast<unsigned>(SPLIT ? c - c0 : c) % STAGES);
             const uint32_t kst = ring_s + s * C::STAGE_BYTES;
             const uint32_t vst = kst + CHUNK * C::RS;
             const int* si = sidx + s * CHUNK;
@@ -284,7 +289,7 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 mnew[j] = fmaxf(mrun[j], mx[j]);
-                alpha[j] = (mnew[j] == -INFINITY) ? 1.f : exp2f(mrun[j] - mnew[j]);
+                alpha[j] = exp2f(mrun[j] - mnew[j]);
                 mrun[j] = mnew[j];
                 lrun[j] *= alpha[j];
             }
@@ -294,8 +299,8 @@ __global__ void __launch_bounds__(WARPS * 32)
                 float p[4];
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    p[j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[mt][j] - mnew[j]);
-                    p[2 + j] = (mnew[j] == -INFINITY) ? 0.f : exp2f(sacc[mt][2 + j] - mnew[j]);
+                    p[j] = exp2f(sacc[mt][j] - mnew[j]);
+                    p[2 + j] = exp2f(sacc[mt][2 + j] - mnew[j]);
                     lrun[j] += p[j] + p[2 + j];
                 }
                 const uint32_t h01 = pack_bf16(p[0], p[1]);
