@@ -165,10 +165,10 @@ def pattern_search(layers, dev, rows=2048, n_f=2):
 
 def attn_traffic():
     """DRAM bytes of one full 200K sparse-attention launch (layer 0 of the warm-up step), from ncu
-    (dram__bytes_read.sum 21.82 GB + dram__bytes_write.sum 1.64 GB; one pass, no replay), taken on
-    the kernel with 32-bit row offsets.  Rows run KV head by KV head, so one head's K/V (102 MB)
-    stays in L2 while its rows gather from it.  Update with the capture when the kernel changes."""
-    return round(21.82e9 + 1.64e9)
+    (dram__bytes_read.sum 22.01 GB + dram__bytes_write.sum 1.64 GB; one pass, no replay), taken on
+    the current kernel.  Rows run KV head by KV head, so one head's K/V (102 MB) stays in L2 while
+    its rows gather from it.  Update with the capture when the kernel changes."""
+    return round(22.01e9 + 1.64e9)
 
 
 def stratified_random_indices(L_, k, dev, seed, rows_per_chunk=8192):
