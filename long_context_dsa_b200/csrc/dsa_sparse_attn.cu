@@ -13,8 +13,9 @@
 //     tokens with 16-byte cp.async into a private multi-stage ring, and
 //     computes on the oldest stage while the younger ones are in flight.
 //     Padding entries (-1) become zero-filled copies that read nothing.
-//     The next chunk's indices are loaded one iteration ahead, so neither
-//     the index load nor a shared producer sits on the critical path.
+//     Indices are read two chunks ahead of their gather and turned into row
+//     offsets one chunk ahead, so neither the index load nor a shared
+//     producer sits on the critical path.
 //   * Online softmax with warp-level bf16 tensor-core MMAs (m16n8k16):
 //     S^T = K_chunk Q^T puts keys on M and the GQA group's query heads on N
 //     (8 columns: no padding at G = 8); O^T += V^T P puts d on M.  P moves
