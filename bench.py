@@ -715,7 +715,7 @@ def run_profile_latent(args):
 
 def run_profile_decode1m(args):
     """One-query fp8 decode indexer at a 1048577-token cache (H_I=64, d_I=128, top-2048) for ncu
-    captures: the split decode kernel writing the row's score keys, then the radix select."""
+    captures: the split decode kernel writing the row's score keys and histogram, then the bin select."""
     import torch
     from long_context_dsa_b200 import dsa, synth
 
@@ -746,7 +746,7 @@ def run_profile_decode1m(args):
 def run_profile_decode(args):
     """One decode indexer call of the batched decode shape for ncu captures: 64 sequences, one
     query each at the end of a 200000-token bf16 key cache (H_I=32, d_I=128, top-2048): the split
-    decode kernel writing every row's score keys, then the radix select."""
+    decode kernel writing every row's score keys and histogram, then the bin select."""
     import torch
     from long_context_dsa_b200 import dsa, synth
 

@@ -399,7 +399,7 @@ int dec_splits(int B, int nkt, int num_sms, int per_sm) {
 }
 
 // Units per SM: more when lengths differ (uneven units balance better); for a few long
-// sequences the merge of their many partial lists would outweigh the finer split.
+// sequences more units per row would add more unit histograms into the same row's bins.
 int per_sm_for(int B, bool varlen) {
     if (varlen) return 6;
     return B >= 32 ? 4 : 2;

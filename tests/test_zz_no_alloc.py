@@ -22,7 +22,7 @@ DEV = "cuda"
 
 # (name, B, n_q, n_kv, H, d, k, fp8): the first has more work tiles than the array's CTA cap; the
 # decode case (one query per sequence at the end of its cache) takes the split decode kernel,
-# whose partial lists and their merge also live in the array
+# whose score keys, histograms and bin-select scratch also live in the array
 CASES = [("h32_k2048_3000", 1, 3000, 3000, 32, 128, 2048, False),
          ("tiny512", 1, 512, 512, 4, 64, 64, False),
          ("fp8_h64_1100", 1, 1100, 1100, 64, 128, 256, True),
