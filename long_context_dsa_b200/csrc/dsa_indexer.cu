@@ -24,7 +24,9 @@
 //   * Epilogue: tcgen05.ld -> ReLU -> x w -> sum over heads -> causal
 //     mask -> admission test against the row's running top-k threshold ->
 //     warp-aggregated append to the row's candidate buffer (global scratch,
-//     L2-resident) -> radix-select prune when the buffer nears capacity.
+//     L2-resident) -> prune when the buffer nears capacity: one histogram pass
+//     keeps a superset of the k best (an exact radix select when ties crowd
+//     one bin), and an exact prune to k ends each row.
 //   * Persistent CTAs take work tiles longest-first in a snake order so the
 //     causal triangle balances across SMs.
 //   * Every wait is bounded (DSA_STATUS_TIMEOUT instead of a hang).
