@@ -357,7 +357,7 @@ def run_gpu(args, rank, world, local_rank):
         "step_roofline": {"t_indexer_s": round(t_idx, 4), "t_gather_s": round(t_gather, 4),
                           "bound_s": round(step_roof_s, 4),
                           "frac": round(step_roof_s / (ms_per_step / 1e3), 4),
-                          "note": "the north star's bound: max(indexer FLOPs at tensor peak, gathered bytes at HBM "
+                          "note": "the step's roofline: max(indexer FLOPs at tensor peak, gathered bytes at HBM "
                                   "peak); the gathered bytes are largely L2 hits here (see roofline), so this bound "
                                   "is not tight and a fraction near 1 does not mean the step is at its limit"},
         "index_sharing": {"all_f_step_ms": round(allf_step, 3), "shared_step_ms": round(ms_per_step, 3),
